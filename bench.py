@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode step on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+copy-on-write block copies (when the workload forks blocks), the KV write of
+this step's tokens, and paged decode attention (partition kernel plus the
+log-sum-exp reduce when a context spans several partitions), all through
+libpa's C ABI on the current CUDA stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|shared_prefix|long|tiny]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, timed on the host cores
+
+Multi-GPU (launched by torch.distributed.run): every rank runs its own
+independent workload (sequences are independent), so per-GPU work is fixed
+(weak scaling); the only collectives are a barrier and a max/sum of timings.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode KV GB/s & fraction of B200 HBM peak; seq-steps/s at 1 GPU"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_TEXT = {
+    "tiny": "tiny: 4+1 seqs, ctx {8,17,34,51,51}, H_q=H_kv=4, D=64, fp16, 32-block pool, 1 CoW fork",
+    "mha": "Llama-2-7B-shaped MHA decode, 1 layer: batch 64, H_q=H_kv=32, D=128, fp16, "
+           "block 16, ctx U[128,2048], pool 1.5x needed",
+    "gqa": "Llama-3-8B-shaped GQA decode, 1 layer: batch 256, H_q=32, H_kv=8, D=128, bf16, "
+           "block 16, ctx lognormal(median 1024, sigma 1) clipped [16,8192]",
+    "shared_prefix": "shared-prefix decode: 100 seqs sharing a 5000-token prefix (312 full blocks + "
+                     "1 partial CoW-forked per seq), suffix U[16,512], H_q=32, H_kv=8, D=128, bf16",
+    "long": "long-context 70B-shaped GQA decode, 1 layer: batch 8, H_q=64, H_kv=8, D=128, bf16, "
+            "ctx U[32768,131072], split-K 512-token partitions + LSE reduce",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mha", choices=list(WORKLOAD_TEXT))
+    ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling only)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition-tokens", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def make_workload(name, batch, seed_offset=0):
+    from paged_kv_cache_391_b200 import workloads as W
+    kw = {}
+    if batch is not None:
+        kw["num_seqs" if name == "shared_prefix" else "batch"] = batch
+    fn = W.CONFIGS[name]
+    import inspect
+    seed = inspect.signature(fn).parameters["seed"].default + 1000 * seed_offset
+    return fn(seed=seed, **kw)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) while
+    the timed region runs."""
+
+    REASONS = {
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.err = [], set(), None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.nv, self.err = None, f"nvml unavailable: {e}"
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, const in self.REASONS.items():
+                    if r & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- CPU (oracle) leg
+
+def oracle_sample(w, target_s: float):
+    """Time the fp64 CPU oracle on a bounded sample of the step: the whole
+    step's cache writes plus decode of a random subset of (sequence, head)
+    rows, sized to take about target_s seconds on every host core. Returns the
+    step-equivalent KV GB/s, seq-steps/s, cores, and a description."""
+    import oracle
+    n_rows = w.num_seqs * w.num_q_heads
+    cores = oracle.num_cores()
+    rng = np.random.default_rng(0)
+    kc, vc = w.k_pool.copy(), w.v_pool.copy()
+
+    def run(rows):
+        t0 = time.perf_counter()
+        if len(w.copy_pairs):
+            oracle.copy_blocks([kc], [vc], w.copy_pairs)
+        oracle.write_kv(w.new_k, w.new_v, kc, vc, w.slot_mapping)
+        oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, w.dtype, rows=rows)
+        return time.perf_counter() - t0
+
+    # calibrate on a few rows, then size the sample
+    order = rng.permutation(n_rows)
+    probe = np.sort(order[:min(n_rows, max(cores, 8))])
+    dt = run(probe)
+    per_row = dt / len(probe)
+    n = int(min(n_rows, max(len(probe), target_s / max(per_row, 1e-9))))
+    rows = np.sort(order[:n])
+    dt = run(rows)
+    # step-equivalent work: the sampled rows' share of the decode
+    row_bytes = (w.context_lens.astype(np.int64)[rows // w.num_q_heads]).sum() * 2 * \
+        w.head_dim * 2 / w.group_size
+    frac_seqs = n / n_rows
+    return {
+        "gbs": row_bytes / dt / 1e9,
+        "seq_steps_per_s": frac_seqs * w.num_seqs / dt,
+        "seconds": dt, "cores": cores,
+        "sample": f"{n} of {n_rows} (seq, q-head) rows of one step, with the step's whole "
+                  f"write_kv/copy_blocks; KV bytes counted per KV head as on the GPU",
+    }
+
+
+# --------------------------------------------------------------------------- GPU leg
+
+def run_gpu(args, rank, world, device):
+    import torch
+    from paged_kv_cache_391_b200 import pa
+
+    w = make_workload(args.workload, args.batch, seed_offset=rank)
+    if args.partition_tokens is not None:
+        w.partition_tokens = args.partition_tokens
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+
+    def dev16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dt).to(device)
+
+    k_cache, v_cache = dev16(w.k_pool), dev16(w.v_pool)
+    q, new_k, new_v = dev16(w.q), dev16(w.new_k), dev16(w.new_v)
+    slots = torch.from_numpy(w.slot_mapping).to(device)
+    pairs = torch.from_numpy(w.copy_pairs).to(device)
+    bt = torch.from_numpy(w.block_tables).to(device)
+    cl = torch.from_numpy(w.context_lens).to(device)
+    out = torch.empty(w.q.shape, dtype=dt, device=device)
+    P = w.partition_tokens
+    ws = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, P, device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    max_ctx = w.max_context_len
+    max_parts = 1 if (P == 0 or max_ctx <= P) else -(-max_ctx // P)
+    launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + \
+        1 + (1 if max_parts > 1 else 0)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(e_dec=None):
+        if pairs.numel():
+            pa.copy_blocks([k_cache], [v_cache], pairs, dev_error=err, stream=stream)
+        pa.write_kv(new_k, new_v, k_cache, v_cache, slots, dev_error=err, stream=stream)
+        if e_dec is not None:
+            e_dec[0].record(stream)
+        pa.decode(out, q, k_cache, v_cache, bt, cl, scale=w.scale, max_context_len=max_ctx,
+                  partition_tokens=P, workspace=ws, dev_error=err, stream=stream)
+        if e_dec is not None:
+            e_dec[1].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    dec_events = [(ev(), ev()) for _ in range(args.steps)]
+    t_start, t_end = ev(), ev()
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        barrier()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(dec_events[i])
+        t_end.record(stream)
+        barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in dec_events]))
+    errors = int(err.item())
+
+    # ---- e2e: host buffers through the public API, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host = {k: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16
+                                    else np.ascontiguousarray(a)).pin_memory()
+                for k, a in (("q", w.q), ("k", w.new_k), ("v", w.new_v),
+                             ("slots", w.slot_mapping), ("bt", w.block_tables),
+                             ("cl", w.context_lens))}
+        out_host = torch.empty(out.shape, dtype=dt).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step():
+            q.view(torch.int16).copy_(host["q"], non_blocking=True)
+            new_k.view(torch.int16).copy_(host["k"], non_blocking=True)
+            new_v.view(torch.int16).copy_(host["v"], non_blocking=True)
+            slots.copy_(host["slots"], non_blocking=True)
+            bt.copy_(host["bt"], non_blocking=True)
+            cl.copy_(host["cl"], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        e2e_ms = a.elapsed_time(b)
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+    return w, elapsed_ms, dec_ms, errors, clocks.report(), e2e, launches_per_step
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return main_reference(args, rank, world)
+
+    import torch
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    w, elapsed_ms, dec_ms, errors, clocks, e2e, launches = run_gpu(args, rank, world, device)
+
+    kv_bytes = w.kv_bytes()
+    sb = w.step_bytes()
+    seqs = w.num_seqs
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([elapsed_ms, e2e["ms"] if e2e else 0.0], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        s = torch.tensor([kv_bytes, seqs, errors], dtype=torch.float64, device=device)
+        dist.all_reduce(s, op=dist.ReduceOp.SUM)
+        elapsed_ms, e2e_max = float(t[0]), float(t[1])
+        if e2e:
+            e2e["ms"] = e2e_max
+        kv_total, seqs_total, errors = float(s[0]), float(s[1]), int(s[2])
+    else:
+        kv_total, seqs_total = float(kv_bytes), float(seqs)
+
+    peak, peak_src = measured_peaks()
+    K = args.steps
+    value = kv_total * K / (elapsed_ms / 1e3) / 1e9
+    dec_achieved = sb["decode"] / (dec_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V, seeded random block placement)",
+        "config": {
+            "workload": WORKLOAD_TEXT[args.workload] if args.batch is None
+            else WORKLOAD_TEXT[args.workload] + f" [batch overridden to {args.batch}]",
+            "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": 16, "partition_tokens": w.partition_tokens,
+            "mean_context_len": float(np.mean(w.context_lens)),
+            "kv_bytes_per_step": kv_bytes,
+            "step": "copy_blocks (if forks) + write_kv + decode (partitions + LSE reduce)",
+            "accumulate": "fp32",
+            "l2": f"inputs larger than L2: {kv_bytes / 1e6:.0f} MB of KV read per step vs "
+                  f"{L2_BYTES / 1e6:.0f} MB L2, no flush" if kv_bytes > 4 * L2_BYTES else
+                  "KV working set fits in L2 (hot-cache number)",
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+        },
+        "seq_steps_per_s": round(seqs_total * K / (elapsed_ms / 1e3), 1),
+        "hbm_frac_of_peak": round(value / peak, 4),
+        "roofline": {
+            "kernel": "pa_decode (decode_partition_kernel + lse_reduce_kernel)",
+            "bound": "hbm",
+            "achieved": round(dec_achieved, 1),
+            "peak": peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(dec_achieved / peak, 4),
+            "algorithmic_bytes_per_launch": sb["decode"],
+            "traffic": None,
+        },
+        "sub_ms": {"decode": round(dec_ms, 5),
+                   "write_kv_and_copies": round(elapsed_ms / K - dec_ms, 5)},
+        "clocks": clocks,
+        "gpu_launches": launches * K,
+        "device_errors": errors,
+    }
+    if e2e:
+        line["e2e"] = {"value": round(kv_total * K / (e2e["ms"] / 1e3) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e["ms"] / K, 5)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(cb["gbs"], 4), "unit": "GB/s", "cores": cb["cores"],
+                                "kind": "oracle", "sample": cb["sample"],
+                                "seq_steps_per_s": round(cb["seq_steps_per_s"], 3),
+                                "seconds": round(cb["seconds"], 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle as it stands, on the host cores,
+    on the same workload, metric and unit. Rank 0 only."""
+    if rank != 0:
+        return 0
+    w = make_workload(args.workload, args.batch)
+    vals, secs = [], []
+    cb = None
+    for _ in range(args.warmup):
+        oracle_sample(w, max(0.5, args.cpu_seconds / 10))
+    for _ in range(args.steps):
+        cb = oracle_sample(w, args.cpu_seconds / max(1, args.steps))
+        vals.append(cb["gbs"])
+        secs.append(cb["seconds"])
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * float(np.mean(secs)), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) q/K/V, seeded random block placement)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "num_seqs": w.num_seqs,
+                   "partition_tokens": w.partition_tokens,
+                   "parallelism": "host threads over (seq, head) rows"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cb["cores"],
+                         "kind": "oracle", "sample": cb["sample"]},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * pa.h -- C ABI of libpa: the paged-KV-cache decode hot path on B200 (sm_100a).
+ *
+ * Three operations of PagedAttention decode, as the pages describe them:
+ *
+ *   pa_write_kv     store this step's new K/V rows in their cache slots
+ *                   ("Optimizing LLM Inference: From PagedAttention to AI
+ *                   Infra", section "Understanding KV Cache ...": K and V of
+ *                   every token are kept at every layer so later steps read
+ *                   them instead of recomputing them).
+ *   pa_decode       single-token decode attention over a paged cache, walking
+ *                   each sequence's block table in logical order (same page,
+ *                   "PagedAttention: Decoupling Logical Context from
+ *                   Contiguous GPU Memory", Figure 2; "The Memory Wall ...",
+ *                   "How it Works Under the Hood" and "Show Me The Code").
+ *                   Long contexts are cut into fixed token partitions whose
+ *                   partial results a log-sum-exp reduce combines (the
+ *                   "sequence splits" of "PagedAttention in Action ...",
+ *                   section "New Developments in 2026").
+ *   pa_copy_blocks  whole-block copies that fork a shared block on
+ *                   copy-on-write ("Optimizing LLM Inference ...",
+ *                   "Copy-on-Write"; "PagedAttention", "KV Cache Sharing
+ *                   (Copy-on-Write)").
+ *
+ * Memory layout (all device memory, row-major, no padding):
+ *   k_cache, v_cache : [num_blocks][num_kv_heads][PA_BLOCK_SIZE][head_dim]
+ *                      16-bit elements (fp16 or bf16), 16-byte aligned base.
+ *   q, out           : [num_seqs][num_q_heads][head_dim]
+ *   k, v (new rows)  : [num_tokens][num_kv_heads][head_dim]
+ *   block_tables     : int32 [num_seqs][block_table_stride]; entry j is the
+ *                      physical block of logical block j (tokens 16j..16j+15).
+ *                      Entries at or past ceil(context_len / 16) are not read.
+ *   context_lens     : int32 [num_seqs], tokens to attend to, including the
+ *                      token written by this step's pa_write_kv.
+ *   slot_mapping     : int64 [num_tokens]; slot = physical_block * 16 + offset;
+ *                      a negative slot marks a padding token and is skipped.
+ *   GQA              : query head h reads KV head h / group_size.
+ *
+ * Ownership: the caller allocates and owns every buffer, the workspace and the
+ * stream. The library borrows the pointers for the duration of the
+ * asynchronous call, allocates no device memory, keeps no per-call state and
+ * never synchronises the stream. Every call is stream-ordered on `stream`
+ * (a cudaStream_t; NULL is the legacy default stream).
+ *
+ * Errors: problems visible on the host (a NULL pointer, an unsupported shape,
+ * a too-small workspace, an out-of-range argument) return a status and launch
+ * nothing. A failed launch returns PA_ERR_CUDA (pa_last_cuda_error() gives
+ * the CUDA error string). Problems only visible in device data (a slot past
+ * the pool, a table entry outside [0, num_blocks), a context length above
+ * max_context_len) never fault and never trap: the offending token or block
+ * is skipped (the context length is clamped to max_context_len) and one is
+ * added to *dev_error when dev_error is not NULL. Device waits are bounded;
+ * a wait that gives up adds PA_DEV_ERR_TIMEOUT to *dev_error.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_BLOCK_SIZE 16
+#define PA_MAX_LAYERS 256
+#define PA_DEV_ERR_TIMEOUT (1 << 24)
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,
+  PA_ERR_UNSUPPORTED = 2,
+  PA_ERR_WORKSPACE_TOO_SMALL = 3,
+  PA_ERR_CUDA = 4
+} pa_status;
+
+typedef enum { PA_DTYPE_F16 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/*
+ * Store num_tokens new K/V rows in the caches: token t goes to slot
+ * slot_mapping[t] of every KV head, i.e. k_cache[slot / 16][h][slot % 16][:]
+ * = k[t][h][:], and the same for v. A bit copy.
+ *   k, v            device, [num_tokens][num_kv_heads][head_dim]
+ *   k_cache, v_cache device, [num_blocks][num_kv_heads][16][head_dim]
+ *   slot_mapping    device int64 [num_tokens]
+ *   block_size      must be 16; head_dim must be a multiple of 8, <= 1024
+ *   dev_error       device int32 counter or NULL (slots >= num_blocks * 16)
+ * num_tokens == 0 is a no-op. Two tokens with the same slot race.
+ */
+pa_status pa_write_kv(const void* k, const void* v, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int32_t num_tokens,
+                      int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                      int64_t num_blocks, pa_dtype dtype, int32_t* dev_error,
+                      void* stream);
+
+/*
+ * Bytes of workspace pa_decode needs for these sizes: fp32 partial outputs
+ * and log-sum-exp values of every (sequence, query head, partition) when a
+ * context spans more than one partition; 0 when no split can happen
+ * (partition_tokens == 0 or max_context_len <= partition_tokens).
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_tokens);
+
+/*
+ * Decode attention of one query token per sequence over its paged context:
+ *   out[s][h] = sum_t softmax_t(scale * <q[s][h], K_t>) V_t,
+ * t over the context_lens[s] tokens the block table of s reaches, K_t and V_t
+ * taken from KV head h / group_size. Accumulation is fp32; out is rounded to
+ * the storage type (round-to-nearest-even). An empty context gives zeros.
+ *   out, q          device, [num_seqs][num_q_heads][head_dim]
+ *   k_cache,v_cache device, [num_blocks][num_q_heads/group_size][16][head_dim]
+ *   block_tables    device int32 [num_seqs][block_table_stride]
+ *   context_lens    device int32 [num_seqs]
+ *   group_size      query heads per KV head: 1..16, divides num_q_heads
+ *   head_dim        64 or 128; block_size must be 16
+ *   max_context_len host upper bound of context_lens (sizes the launch)
+ *   partition_tokens 0 = one partition per sequence; else a multiple of 16:
+ *                   contexts longer than it are split into partitions of
+ *                   that many tokens, reduced by log-sum-exp
+ *   workspace       device, >= pa_decode_workspace_size(...) bytes, 256-byte
+ *                   aligned; may be NULL when that size is 0
+ *   dev_error       device int32 counter or NULL
+ * Deterministic: no atomics in the arithmetic; the result depends only on the
+ * logical order of tokens, not on which physical blocks hold them.
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t block_table_stride,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t group_size, int32_t head_dim, int32_t block_size,
+                    int64_t num_blocks, int32_t max_context_len, float scale,
+                    int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_error, pa_dtype dtype, void* stream);
+
+/*
+ * Copy-on-write block copies: for each pair p and each layer l,
+ * k_caches[l][dst] = k_caches[l][src] and v_caches[l][dst] = v_caches[l][src]
+ * (whole blocks: num_kv_heads * 16 * head_dim elements), src = mapping[2p],
+ * dst = mapping[2p+1].
+ *   k_caches, v_caches HOST arrays of num_layers DEVICE pointers
+ *   block_mapping   device int64 [num_pairs][2]
+ *   num_layers      1..PA_MAX_LAYERS
+ *   dev_error       device int32 counter or NULL (pairs outside [0, num_blocks))
+ * A dst that repeats, or that is also some pair's src, is undefined.
+ */
+pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_layers,
+                         const int64_t* block_mapping, int32_t num_pairs,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         int64_t num_blocks, pa_dtype dtype, int32_t* dev_error,
+                         void* stream);
+
+/* Static description of a status code. */
+const char* pa_status_string(pa_status status);
+
+/* The CUDA error string of the last PA_ERR_CUDA on this thread ("" if none). */
+const char* pa_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

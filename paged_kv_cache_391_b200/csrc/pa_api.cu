@@ -1,0 +1,213 @@
+// pa_api.cu -- libpa's C ABI (declared in include/pa.h): argument checks,
+// launch geometry, workspace sizing and TMA descriptor encoding. Allocates
+// no device memory and never synchronises the caller's stream.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+pa_status cuda_fail(cudaError_t e) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return PA_ERR_CUDA;
+}
+
+pa_status driver_fail(const char* what, int code) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s failed (CUresult %d)", what, code);
+  return PA_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_dtype(pa_dtype d) { return d == PA_DTYPE_F16 || d == PA_DTYPE_BF16; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The cache pool [NB][H_kv][16][D] as a 4-D tensor (D innermost); a box is
+// 64 columns x 16 slots of one (block, KV head), landing as 16 rows of 128
+// bytes with the 128-byte swizzle.
+pa_status encode_pool_map(CUtensorMap* map, const void* pool, int64_t num_blocks,
+                          int32_t num_kv_heads, int32_t head_dim, pa_dtype dtype) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return driver_fail("cuTensorMapEncodeTiled lookup", -1);
+  const cuuint64_t row = (cuuint64_t)head_dim * 2;
+  cuuint64_t dims[4] = {(cuuint64_t)head_dim, PA_BLOCK_SIZE, (cuuint64_t)num_kv_heads,
+                        (cuuint64_t)num_blocks};
+  cuuint64_t strides[3] = {row, row * PA_BLOCK_SIZE, row * PA_BLOCK_SIZE * num_kv_heads};
+  cuuint32_t box[4] = {64, PA_BLOCK_SIZE, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(map,
+                      dtype == PA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                      4, const_cast<void*>(pool), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return driver_fail("cuTensorMapEncodeTiled", (int)r);
+  return PA_OK;
+}
+
+int64_t max_partitions(int32_t max_context_len, int32_t partition_tokens) {
+  if (partition_tokens <= 0 || max_context_len <= partition_tokens) return 1;
+  return ((int64_t)max_context_len + partition_tokens - 1) / partition_tokens;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case PA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case PA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* pa_last_cuda_error(void) { return g_last_cuda_error; }
+
+pa_status pa_write_kv(const void* k, const void* v, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, int64_t num_blocks, pa_dtype dtype,
+                      int32_t* dev_error, void* stream) {
+  if (num_tokens < 0 || num_kv_heads < 1 || num_blocks < 1 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != PA_BLOCK_SIZE || head_dim < 8 || head_dim > 1024 || head_dim % 8)
+    return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8) || (dev_error && !aligned(dev_error, 4)))
+    return PA_ERR_INVALID_ARG;
+  cudaError_t e = pa::launch_write_kv(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                      num_kv_heads, head_dim, num_blocks, dev_error,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const int64_t parts = max_partitions(max_context_len, partition_tokens);
+  if (parts <= 1) return 0;
+  const size_t rows = (size_t)num_seqs * num_q_heads * parts;
+  return round256(rows * head_dim * sizeof(float)) + round256(rows * sizeof(float));
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t block_table_stride,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t group_size, int32_t head_dim, int32_t block_size,
+                    int64_t num_blocks, int32_t max_context_len, float scale,
+                    int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_error, pa_dtype dtype, void* stream) {
+  if (num_seqs < 0 || num_q_heads < 1 || group_size < 1 || num_blocks < 1 ||
+      max_context_len < 0 || partition_tokens < 0 || !valid_dtype(dtype) || !isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != PA_BLOCK_SIZE || (head_dim != 64 && head_dim != 128) || group_size > 16 ||
+      num_q_heads % group_size != 0 || partition_tokens % PA_BLOCK_SIZE != 0)
+    return PA_ERR_UNSUPPORTED;
+  const int32_t num_kv_heads = num_q_heads / group_size;
+  if (num_seqs > 65535 || num_kv_heads > 65535 || num_blocks > (int64_t(1) << 32))
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || (dev_error && !aligned(dev_error, 4)))
+    return PA_ERR_INVALID_ARG;
+  const int64_t max_blocks = ((int64_t)max_context_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE;
+  if (block_table_stride < max_blocks || block_table_stride < 1) return PA_ERR_INVALID_ARG;
+
+  const int64_t parts = max_partitions(max_context_len, partition_tokens);
+  if (parts > 0x7fffffff) return PA_ERR_UNSUPPORTED;
+  const size_t need =
+      pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens);
+  if (need > 0) {
+    if (!workspace || !aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
+  }
+
+  pa::DecodeLaunch a;
+  pa_status st = encode_pool_map(&a.tm_k, k_cache, num_blocks, num_kv_heads, head_dim, dtype);
+  if (st != PA_OK) return st;
+  st = encode_pool_map(&a.tm_v, v_cache, num_blocks, num_kv_heads, head_dim, dtype);
+  if (st != PA_OK) return st;
+  const size_t rows = (size_t)num_seqs * num_q_heads * parts;
+  a.out = out;
+  a.part_o = need ? static_cast<float*>(workspace) : nullptr;
+  a.part_lse = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                               round256(rows * head_dim * sizeof(float)))
+                    : nullptr;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.bt_stride = block_table_stride;
+  a.context_lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group_size;
+  a.head_dim = head_dim;
+  a.num_blocks = num_blocks;
+  a.max_context_len = max_context_len;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
+  a.part_tokens = parts > 1 ? partition_tokens : (int32_t)(max_blocks * PA_BLOCK_SIZE);
+  a.part_blocks = parts > 1 ? partition_tokens / PA_BLOCK_SIZE : (int32_t)(max_blocks > 0 ? max_blocks : 1);
+  if (a.part_tokens < PA_BLOCK_SIZE) a.part_tokens = PA_BLOCK_SIZE;
+  a.max_parts = (int32_t)parts;
+  a.dev_error = dev_error;
+  a.bf16 = dtype == PA_DTYPE_BF16;
+  cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_layers,
+                         const int64_t* block_mapping, int32_t num_pairs, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                         pa_dtype dtype, int32_t* dev_error, void* stream) {
+  if (num_layers < 1 || num_pairs < 0 || num_kv_heads < 1 || num_blocks < 1 ||
+      !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_layers > PA_MAX_LAYERS || block_size != PA_BLOCK_SIZE || head_dim < 8 ||
+      head_dim % 8)
+    return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_caches || !v_caches || !block_mapping || !aligned(block_mapping, 8) ||
+      (dev_error && !aligned(dev_error, 4)))
+    return PA_ERR_INVALID_ARG;
+  for (int l = 0; l < num_layers; ++l)
+    if (!k_caches[l] || !v_caches[l] || !aligned(k_caches[l], 16) || !aligned(v_caches[l], 16))
+      return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes = (int64_t)num_kv_heads * PA_BLOCK_SIZE * head_dim * 2;
+  cudaError_t e = pa::launch_copy_blocks(k_caches, v_caches, num_layers, block_mapping, num_pairs,
+                                         block_bytes, num_blocks, dev_error,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

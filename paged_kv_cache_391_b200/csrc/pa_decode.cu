@@ -1,0 +1,490 @@
+// pa_decode.cu -- paged single-token decode attention for sm_100a.
+//
+// What it computes ("Optimizing LLM Inference: From PagedAttention to AI
+// Infra", "PagedAttention: Decoupling Logical Context from Contiguous GPU
+// Memory", Figure 2; "The Memory Wall ...", "How it Works Under the Hood" and
+// "Show Me The Code"): for every sequence s and query head h,
+//     out[s][h] = sum_t softmax_t(scale * <q[s][h], K_t>) V_t
+// over the context's tokens, found by walking the block table in logical
+// order. Long contexts are split into fixed token partitions ("PagedAttention
+// in Action ...", "New Developments in 2026": sequence splits as a unit of
+// decode scheduling) whose results a log-sum-exp reduce combines.
+//
+// Design (B200):
+//  * One CTA per (partition, KV head, sequence); its four warps take the
+//    partition's 16-token blocks round-robin, each with a private 3-stage ring
+//    of shared-memory tiles. A tile (one block, one KV head: 16 x D values,
+//    contiguous in HBM) arrives by TMA as 64-column boxes with a 128-byte
+//    swizzle, so the ldmatrix reads below are bank-conflict free. Completion
+//    is tracked by one mbarrier per stage; every wait is bounded.
+//  * All query heads of a KV head share each K/V load (GQA). q.K^T and P.V
+//    run on the tensor cores as m16n8k16 tiles with the query heads as the M
+//    dimension (up to 16), tokens and head-dim columns as N and K; the P tile
+//    is taken straight from the q.K^T accumulators without a shuffle.
+//  * Softmax is online, per warp, in fp32 and base 2 (scale * log2 e folded
+//    into one multiply); the four warps and then the partitions are merged by
+//    log-sum-exp. Tokens past the context are masked to -inf and their V rows
+//    zeroed in shared memory, so stale cache contents never reach the output.
+//  * The arithmetic follows logical token order only, so the output does not
+//    depend on which physical blocks hold the context, bit for bit.
+#include <math.h>
+
+#include "pa.h"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+constexpr int kBlockTokens = 16;
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+struct DecodeSmem {
+  static constexpr int kStages = 3;
+  static constexpr int kSubTiles = D / 64;                 // 128-byte TMA boxes per tile
+  static constexpr int kTileBytes = kBlockTokens * D * 2;  // K (or V) of one block, one KV head
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kWarpBytes = kStages * kStageBytes;
+  static constexpr int kTileRegion = kWarps * kWarpBytes;
+  static constexpr int kBarOffset = kTileRegion;
+  static constexpr int kBytes = kTileRegion + kWarps * kStages * 8;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+  static constexpr int kMergeStride = D + 8;    // floats per (warp, head) row of the merge
+  static_assert(kWarps * 16 * kMergeStride * 4 + 2 * kWarps * 16 * 4 <= kTileRegion,
+                "merge scratch must fit in the tile region");
+};
+
+// Byte offset of element (token t, column d) inside one swizzled tile: the
+// tile is D/64 boxes of 16 rows x 128 bytes, and the 16-byte chunk index
+// within a row is XORed with (row % 8), as TMA's 128-byte swizzle lays it out.
+__device__ __forceinline__ uint32_t tile_off(int t, int d) {
+  return (uint32_t)((d >> 6) * 2048 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4) + (d & 7) * 2);
+}
+
+template <typename T, int D, bool kTwoRows>
+__global__ void __launch_bounds__(kThreads)
+    decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, T* __restrict__ out,
+                            float* __restrict__ part_o, float* __restrict__ part_lse,
+                            const T* __restrict__ q, const int32_t* __restrict__ block_tables,
+                            int bt_stride, const int32_t* __restrict__ context_lens,
+                            int num_q_heads, int group, int64_t num_blocks, int max_context_len,
+                            float scale_log2, int part_blocks, int max_parts,
+                            int32_t* __restrict__ dev_error) {
+  using SM = DecodeSmem<D>;
+  using E = Elem<T>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOffset);
+
+  const int part = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+
+  int L = context_lens[seq];
+  if (L < 0 || L > max_context_len) {
+    if (part == 0 && kvh == 0 && tid == 0 && dev_error) atomicAdd(dev_error, 1);
+    L = L < 0 ? 0 : max_context_len;
+  }
+  const int nblk_seq = (L + kBlockTokens - 1) / kBlockTokens;
+  const int n_parts = nblk_seq > 0 ? (nblk_seq + part_blocks - 1) / part_blocks : 1;
+  if (part >= n_parts) return;
+  const int blk_begin = part * part_blocks;
+  const int nblk = min(nblk_seq - blk_begin, part_blocks);  // 0 only for an empty context
+  const int q_head0 = kvh * group;
+
+  // ---- this warp's share: blocks blk_begin + warp + kWarps * it
+  const int n_mine = nblk > warp ? (nblk - warp + kWarps - 1) / kWarps : 0;
+  uint8_t* wtiles = smem + warp * SM::kWarpBytes;
+  uint64_t* wbars = bars + warp * SM::kStages;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < SM::kStages; ++s) mbar_init(&wbars[s], 1);
+    fence_barrier_init();
+    if (warp == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+  }
+  __syncwarp();
+
+  // Physical block ids, 32 iterations per register window; ids outside the
+  // pool are counted once (by the KV-head-0 CTA) and skipped.
+  const int32_t* bt_mine = block_tables + (size_t)seq * bt_stride + blk_begin + warp;
+  auto load_pid = [&](int it) -> int {
+    int p = -1;
+    if (it < n_mine) {
+      p = __ldg(bt_mine + kWarps * it);
+      if (p < 0 || p >= num_blocks) {
+        if (kvh == 0 && dev_error) atomicAdd(dev_error, 1);
+        p = -1;
+      }
+    }
+    return p;
+  };
+  int win = 0;
+  int pid_cur = load_pid(lane);
+  int pid_nxt = load_pid(32 + lane);
+  auto pid_of = [&](int it) -> int {
+    const int v = ((it >> 5) == win) ? pid_cur : pid_nxt;
+    return __shfl_sync(kFull, v, it & 31);
+  };
+  auto issue = [&](int it, int p) {  // lane 0 only
+    const int st = it % SM::kStages;
+    uint8_t* kt = wtiles + st * SM::kStageBytes;
+    uint8_t* vt = kt + SM::kTileBytes;
+    if (p >= 0) {
+      mbar_arrive_expect_tx(&wbars[st], 2 * SM::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < SM::kSubTiles; ++c) {
+        tma_load_4d(kt + c * 2048, &tm_k, &wbars[st], c * 64, 0, kvh, p);
+        tma_load_4d(vt + c * 2048, &tm_v, &wbars[st], c * 64, 0, kvh, p);
+      }
+    } else {
+      mbar_arrive(&wbars[st]);  // nothing to load: complete the phase empty
+    }
+  };
+  {
+    const int n_pro = min(n_mine, SM::kStages);
+    for (int it = 0; it < n_pro; ++it) {
+      const int p = pid_of(it);
+      if (lane == 0) issue(it, p);
+    }
+  }
+
+  // ---- query fragments (A operand of q.K^T): rows = heads of this group
+  uint32_t qa[D / 16][4];
+  {
+    const uint32_t* qa_row =
+        gid < group ? reinterpret_cast<const uint32_t*>(
+                          q + ((size_t)seq * num_q_heads + q_head0 + gid) * D)
+                    : nullptr;
+    const uint32_t* qb_row =
+        (kTwoRows && gid + 8 < group)
+            ? reinterpret_cast<const uint32_t*>(q + ((size_t)seq * num_q_heads + q_head0 + gid + 8) * D)
+            : nullptr;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qa[kk][0] = qa_row ? __ldg(qa_row + kk * 8 + tig) : 0u;
+      qa[kk][1] = qb_row ? __ldg(qb_row + kk * 8 + tig) : 0u;
+      qa[kk][2] = qa_row ? __ldg(qa_row + kk * 8 + 4 + tig) : 0u;
+      qa[kk][3] = qb_row ? __ldg(qb_row + kk * 8 + 4 + tig) : 0u;
+    }
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+
+  const int mi = lane >> 3, r8 = lane & 7;
+  int it = 0;
+  bool timed_out = false;
+  for (; it < n_mine; ++it) {
+    if (it > 0 && (it & 31) == 0) {
+      ++win;
+      pid_cur = pid_nxt;
+      pid_nxt = load_pid((win + 1) * 32 + lane);
+    }
+    const int st = it % SM::kStages;
+    const uint32_t parity = (uint32_t)((it / SM::kStages) & 1);
+    const int p = pid_of(it);
+    if (!__all_sync(kFull, mbar_wait(&wbars[st], parity))) {
+      timed_out = true;
+      break;
+    }
+    if (p >= 0) {
+      uint8_t* kt = wtiles + st * SM::kStageBytes;
+      uint8_t* vt = kt + SM::kTileBytes;
+      const int j = blk_begin + warp + kWarps * it;
+      const int valid = min(kBlockTokens, L - j * kBlockTokens);
+      if (valid < kBlockTokens) {
+        // Zero the V rows past the context: P is 0 there, and 0 * NaN would not be.
+        const int nrow = kBlockTokens - valid;
+        for (int i = lane; i < nrow * SM::kSubTiles * 8; i += 32) {
+          const int c = i / (nrow * 8), rem = i % (nrow * 8);
+          *reinterpret_cast<uint4*>(vt + c * 2048 + (valid + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+
+      // S = Q K^T for the 16 tokens: two n-tiles of 8 tokens, K over D.
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t kbase = smem_addr(kt);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbase + tile_off((mi >> 1) * 8 + r8, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+        E::mma(s0, qa[kk], b0, b1);
+        E::mma(s1, qa[kk], b2, b3);
+      }
+
+      // Online softmax (base 2). Lane holds, for head row a = gid (and
+      // b = gid + 8), tokens 2tig, 2tig+1 (s0) and 8+2tig, 9+2tig (s1).
+      const int t0 = 2 * tig;
+      const bool v0 = t0 < valid, v1 = t0 + 1 < valid, v2 = t0 + 8 < valid, v3 = t0 + 9 < valid;
+      uint32_t pa[4];
+      {
+        const float x0 = v0 ? s0[0] * scale_log2 : -INFINITY;
+        const float x1 = v1 ? s0[1] * scale_log2 : -INFINITY;
+        const float x2 = v2 ? s1[0] * scale_log2 : -INFINITY;
+        const float x3 = v3 ? s1[1] * scale_log2 : -INFINITY;
+        float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const float m_new = fmaxf(m_a, mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = exp2f(m_a - m_use);
+        pa[0] = E::pack(exp2f(x0 - m_use), exp2f(x1 - m_use));
+        pa[2] = E::pack(exp2f(x2 - m_use), exp2f(x3 - m_use));
+        const float2 u0 = E::unpack(pa[0]), u2 = E::unpack(pa[2]);
+        l_a = l_a * alpha + ((u0.x + u0.y) + (u2.x + u2.y));
+        m_a = m_new;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] *= alpha;
+          o[n][1] *= alpha;
+        }
+      }
+      if (kTwoRows) {
+        const float x0 = v0 ? s0[2] * scale_log2 : -INFINITY;
+        const float x1 = v1 ? s0[3] * scale_log2 : -INFINITY;
+        const float x2 = v2 ? s1[2] * scale_log2 : -INFINITY;
+        const float x3 = v3 ? s1[3] * scale_log2 : -INFINITY;
+        float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const float m_new = fmaxf(m_b, mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = exp2f(m_b - m_use);
+        pa[1] = E::pack(exp2f(x0 - m_use), exp2f(x1 - m_use));
+        pa[3] = E::pack(exp2f(x2 - m_use), exp2f(x3 - m_use));
+        const float2 u1 = E::unpack(pa[1]), u3 = E::unpack(pa[3]);
+        l_b = l_b * alpha + ((u1.x + u1.y) + (u3.x + u3.y));
+        m_b = m_new;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][2] *= alpha;
+          o[n][3] *= alpha;
+        }
+      } else {
+        pa[1] = 0u;
+        pa[3] = 0u;
+      }
+
+      // O += P V: N = head-dim columns (pairs of 8-column n-tiles), K = 16 tokens.
+      const uint32_t vbase = smem_addr(vt);
+#pragma unroll
+      for (int n2 = 0; n2 < D / 16; ++n2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(vbase + tile_off((mi & 1) * 8 + r8, n2 * 16 + (mi >> 1) * 8), b0, b1, b2,
+                      b3);
+        E::mma(o[2 * n2], pa, b0, b1);
+        E::mma(o[2 * n2 + 1], pa, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (it + SM::kStages < n_mine) {
+      const int pn = pid_of(it + SM::kStages);
+      if (lane == 0) issue(it + SM::kStages, pn);
+    }
+  }
+  if (timed_out) {
+    // Let the copies already in flight land (each wait bounded) before the
+    // shared memory is reused or the CTA exits, then report.
+    const int last = min(n_mine, it + SM::kStages);
+    for (int k = it; k < last; ++k) (void)mbar_wait(&wbars[k % SM::kStages], (k / SM::kStages) & 1);
+    if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
+  }
+
+  // ---- merge the four warps (log-sum-exp), then write out or the partials
+  l_a += __shfl_xor_sync(kFull, l_a, 1);
+  l_a += __shfl_xor_sync(kFull, l_a, 2);
+  if (kTwoRows) {
+    l_b += __shfl_xor_sync(kFull, l_b, 1);
+    l_b += __shfl_xor_sync(kFull, l_b, 2);
+  }
+  __syncthreads();  // every warp is done with its tiles
+  float* mo = reinterpret_cast<float*>(smem);
+  float* mm = mo + kWarps * 16 * SM::kMergeStride;
+  float* ml = mm + kWarps * 16;
+  if (gid < group) {
+    float* row = mo + (warp * 16 + gid) * SM::kMergeStride;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n)
+      *reinterpret_cast<float2*>(row + n * 8 + 2 * tig) = make_float2(o[n][0], o[n][1]);
+    if (tig == 0) {
+      mm[warp * 16 + gid] = m_a;
+      ml[warp * 16 + gid] = l_a;
+    }
+  }
+  if (kTwoRows && gid + 8 < group) {
+    float* row = mo + (warp * 16 + gid + 8) * SM::kMergeStride;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n)
+      *reinterpret_cast<float2*>(row + n * 8 + 2 * tig) = make_float2(o[n][2], o[n][3]);
+    if (tig == 0) {
+      mm[warp * 16 + gid + 8] = m_b;
+      ml[warp * 16 + gid + 8] = l_b;
+    }
+  }
+  __syncthreads();
+
+  const bool direct = n_parts == 1;
+  for (int idx = tid; idx < group * (D / 4); idx += kThreads) {
+    const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * 16 + h]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float sc = exp2f(mm[w * 16 + h] - M);
+        lsum += ml[w * 16 + h] * sc;
+        const float4 v = *reinterpret_cast<const float4*>(mo + (w * 16 + h) * SM::kMergeStride + d);
+        acc.x += sc * v.x;
+        acc.y += sc * v.y;
+        acc.z += sc * v.z;
+        acc.w += sc * v.w;
+      }
+    }
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lsum > 0.f) {
+      res.x = acc.x / lsum;
+      res.y = acc.y / lsum;
+      res.z = acc.z / lsum;
+      res.w = acc.w / lsum;
+    }
+    const size_t orow = (size_t)seq * num_q_heads + q_head0 + h;
+    if (direct) {
+      uint2 pk;
+      pk.x = E::pack(res.x, res.y);
+      pk.y = E::pack(res.z, res.w);
+      *reinterpret_cast<uint2*>(out + orow * D + d) = pk;
+    } else {
+      *reinterpret_cast<float4*>(part_o + (orow * max_parts + part) * D + d) = res;
+      if (d == 0) part_lse[orow * max_parts + part] = lsum > 0.f ? M + log2f(lsum) : -INFINITY;
+    }
+  }
+}
+
+// Combine the partitions of one (sequence, query head): weights
+// 2^(lse_p - max lse), normalised; fixed summation order (deterministic).
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    lse_reduce_kernel(T* __restrict__ out, const float* __restrict__ part_o,
+                      const float* __restrict__ part_lse, const int32_t* __restrict__ context_lens,
+                      int num_q_heads, int max_context_len, int part_tokens, int max_parts) {
+  constexpr int kW = 8;
+  constexpr int kLanes = D / 4;            // float4 columns per partition row
+  constexpr int kRowsPerWarp = 32 / kLanes;
+  constexpr int kStreams = kW * kRowsPerWarp;
+  using E = Elem<T>;
+  const int hq = blockIdx.x, seq = blockIdx.y;
+  int L = context_lens[seq];
+  L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
+  const int n = (L + part_tokens - 1) / part_tokens;
+  if (n <= 1) return;  // written directly by the partition kernel
+  const size_t row = (size_t)seq * num_q_heads + hq;
+  const float* lse = part_lse + row * max_parts;
+  const float4* po = reinterpret_cast<const float4*>(part_o + row * max_parts * D);
+  __shared__ float red[kW];
+  __shared__ float4 acc_s[kStreams][kLanes];
+  __shared__ float ws_s[kStreams];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+
+  float M = -INFINITY;
+  for (int p = tid; p < n; p += kW * 32) M = fmaxf(M, lse[p]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  if (lane == 0) red[w] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int i = 1; i < kW; ++i) M = fmaxf(M, red[i]);
+
+  const int stream = w * kRowsPerWarp + lane / kLanes;
+  const int c = lane % kLanes;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float ws = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int p = stream; p < n; p += kStreams) {
+      const float wt = exp2f(lse[p] - M);
+      const float4 v = po[(size_t)p * kLanes + c];
+      ws += wt;
+      acc.x += wt * v.x;
+      acc.y += wt * v.y;
+      acc.z += wt * v.z;
+      acc.w += wt * v.w;
+    }
+  }
+  acc_s[stream][c] = acc;
+  if (c == 0) ws_s[stream] = ws;
+  __syncthreads();
+  if (tid < kLanes) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kStreams; ++i) {
+      const float4 v = acc_s[i][tid];
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+      s += ws_s[i];
+    }
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s > 0.f) {
+      res.x = a.x / s;
+      res.y = a.y / s;
+      res.z = a.z / s;
+      res.w = a.w / s;
+    }
+    uint2 pk;
+    pk.x = E::pack(res.x, res.y);
+    pk.y = E::pack(res.z, res.w);
+    *reinterpret_cast<uint2*>(out + row * D + tid * 4) = pk;
+  }
+}
+
+template <typename T, int D, bool kTwoRows>
+static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
+  using SM = DecodeSmem<D>;
+  auto kern = decode_partition_kernel<T, D, kTwoRows>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.max_parts, a.num_kv_heads, a.num_seqs);
+  kern<<<grid, kThreads, SM::kAlloc, stream>>>(
+      a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, static_cast<const T*>(a.q),
+      a.block_tables, a.bt_stride, a.context_lens, a.num_q_heads, a.group, a.num_blocks,
+      a.max_context_len, a.scale_log2, a.part_blocks, a.max_parts, a.dev_error);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.max_parts <= 1) return e;
+  dim3 rgrid(a.num_q_heads, a.num_seqs);
+  lse_reduce_kernel<T, D><<<rgrid, 256, 0, stream>>>(
+      static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.num_q_heads,
+      a.max_context_len, a.part_tokens, a.max_parts);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_dtype(const DecodeLaunch& a, cudaStream_t stream) {
+  const bool two = a.group > 8;
+  if (a.head_dim == 128)
+    return two ? launch_typed<T, 128, true>(a, stream) : launch_typed<T, 128, false>(a, stream);
+  return two ? launch_typed<T, 64, true>(a, stream) : launch_typed<T, 64, false>(a, stream);
+}
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
+  return a.bf16 ? launch_dtype<__nv_bfloat16>(a, stream) : launch_dtype<__half>(a, stream);
+}
+
+}  // namespace pa

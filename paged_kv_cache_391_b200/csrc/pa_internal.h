@@ -1,0 +1,49 @@
+// pa_internal.h -- launch interfaces between libpa's C ABI (pa_api.cu) and
+// its kernel translation units. Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pa {
+
+struct DecodeLaunch {
+  CUtensorMap tm_k;  // K pool as [NB][H_kv][16][D], 64x16 boxes, 128-byte swizzle
+  CUtensorMap tm_v;
+  void* out;
+  float* part_o;     // [S][H_q][max_parts][D]
+  float* part_lse;   // [S][H_q][max_parts]
+  const void* q;
+  const int32_t* block_tables;
+  int32_t bt_stride;
+  const int32_t* context_lens;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t group;
+  int32_t head_dim;
+  int64_t num_blocks;
+  int32_t max_context_len;
+  float scale_log2;  // scale * log2(e)
+  int32_t part_blocks;
+  int32_t part_tokens;
+  int32_t max_parts;
+  int32_t* dev_error;
+  int bf16;          // 0 = fp16, 1 = bf16
+};
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+
+cudaError_t launch_write_kv(const void* k, const void* v, void* k_cache, void* v_cache,
+                            const int64_t* slot_mapping, int32_t num_tokens,
+                            int32_t num_kv_heads, int32_t head_dim, int64_t num_blocks,
+                            int32_t* dev_error, cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_layers,
+                               const int64_t* block_mapping, int32_t num_pairs,
+                               int64_t block_bytes, int64_t num_blocks, int32_t* dev_error,
+                               cudaStream_t stream);
+
+}  // namespace pa

@@ -1,0 +1,173 @@
+"""Thin ctypes binding of libpa (include/pa.h): argument marshalling only.
+
+Every step of the hot path runs in libpa's CUDA kernels. PyTorch supplies
+device memory and the current stream. If libpa.so is missing, every call
+raises -- there is no CPU or eager fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA = range(5)
+PA_DTYPE_F16, PA_DTYPE_BF16 = 0, 1
+PA_BLOCK_SIZE = 16
+PA_MAX_LAYERS = 256
+PA_DEV_ERR_TIMEOUT = 1 << 24
+
+# Every entry point include/pa.h declares.
+EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_blocks",
+           "pa_status_string", "pa_last_cuda_error")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = f"{where}: {status_string(status)}"
+        if status == PA_ERR_CUDA:
+            msg += f" ({last_cuda_error()})"
+        super().__init__(msg)
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Open libpa.so (once). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_391_b200.build` "
+                    "(or __graft_entry__.build()); there is no fallback path")
+            L = ctypes.CDLL(LIB_PATH)
+            P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+            L.pa_write_kv.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i64, ctypes.c_int, P, P]
+            L.pa_write_kv.restype = ctypes.c_int
+            L.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+            L.pa_decode_workspace_size.restype = sz
+            L.pa_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, i32,
+                                    ctypes.c_float, i32, P, sz, P, ctypes.c_int, P]
+            L.pa_decode.restype = ctypes.c_int
+            L.pa_copy_blocks.argtypes = [P, P, i32, P, i32, i32, i32, i32, i64, ctypes.c_int, P, P]
+            L.pa_copy_blocks.restype = ctypes.c_int
+            L.pa_status_string.argtypes = [ctypes.c_int]
+            L.pa_status_string.restype = ctypes.c_char_p
+            L.pa_last_cuda_error.argtypes = []
+            L.pa_last_cuda_error.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().pa_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> str:
+    return lib().pa_last_cuda_error().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_DTYPE_F16
+    if t.dtype == torch.bfloat16:
+        return PA_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: fp16 or bf16 only")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libpa must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def write_kv(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+             slot_mapping: torch.Tensor, *, dev_error: torch.Tensor | None = None,
+             stream=None) -> None:
+    """Store new rows k, v ``[T, H_kv, D]`` in the caches ``[NB, H_kv, 16, D]`` at
+    ``slot_mapping`` (int64 ``[T]``)."""
+    T, H, D = k.shape
+    NB = k_cache.shape[0]
+    assert v.shape == k.shape and k_cache.shape == v_cache.shape == (NB, H, PA_BLOCK_SIZE, D)
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.numel() == T
+    assert k.dtype == v.dtype == k_cache.dtype == v_cache.dtype
+    st = lib().pa_write_kv(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                           T, H, D, PA_BLOCK_SIZE, NB, _dtype_code(k), _ptr(dev_error),
+                           _stream(stream, k_cache.device))
+    _check(st, "pa_write_kv")
+
+
+def decode_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                          partition_tokens: int) -> int:
+    return int(lib().pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                              partition_tokens))
+
+
+def alloc_workspace(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens,
+                    device) -> torch.Tensor | None:
+    n = decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           block_tables: torch.Tensor, context_lens: torch.Tensor, *, scale: float,
+           max_context_len: int, partition_tokens: int = 512,
+           workspace: torch.Tensor | None = None, dev_error: torch.Tensor | None = None,
+           stream=None) -> torch.Tensor:
+    """Paged decode attention: ``out [S, H_q, D] = attention(q, paged K/V)``."""
+    S, Hq, D = q.shape
+    NB, Hkv = k_cache.shape[:2]
+    assert out.shape == q.shape and out.dtype == q.dtype == k_cache.dtype == v_cache.dtype
+    assert k_cache.shape == v_cache.shape == (NB, Hkv, PA_BLOCK_SIZE, D)
+    assert block_tables.dtype == torch.int32 and block_tables.dim() == 2
+    assert context_lens.dtype == torch.int32 and context_lens.numel() == S
+    if Hq % Hkv:
+        raise ValueError("num_q_heads must be a multiple of num_kv_heads")
+    if workspace is None:
+        workspace = alloc_workspace(S, Hq, D, max_context_len, partition_tokens, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                         block_tables.shape[1], _ptr(context_lens), S, Hq, Hq // Hkv, D,
+                         PA_BLOCK_SIZE, NB, int(max_context_len), float(scale),
+                         int(partition_tokens), _ptr(workspace), ws_bytes, _ptr(dev_error),
+                         _dtype_code(q), _stream(stream, q.device))
+    _check(st, "pa_decode")
+    return out
+
+
+def copy_blocks(k_caches, v_caches, block_mapping: torch.Tensor, *,
+                dev_error: torch.Tensor | None = None, stream=None) -> None:
+    """Copy whole blocks ``src -> dst`` (int64 ``[n, 2]`` on the device) in every
+    layer's K and V cache (lists of ``[NB, H_kv, 16, D]`` tensors)."""
+    L = len(k_caches)
+    assert L == len(v_caches) and L >= 1
+    NB, H, bs, D = k_caches[0].shape
+    assert block_mapping.dtype == torch.int64
+    n = block_mapping.numel() // 2
+    kp = (ctypes.c_void_p * L)(*[_ptr(c) for c in k_caches])
+    vp = (ctypes.c_void_p * L)(*[_ptr(c) for c in v_caches])
+    st = lib().pa_copy_blocks(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
+                              L, _ptr(block_mapping), n, H, D, bs, NB,
+                              _dtype_code(k_caches[0]), _ptr(dev_error),
+                              _stream(stream, k_caches[0].device))
+    _check(st, "pa_copy_blocks")
