@@ -134,9 +134,10 @@ def test_shared_blocks_equal_private_copies_bitwise():
     d = DeviceStep(w).step()
     # give every sequence private copies of the shared full prefix blocks
     full = 600 // 16
-    kc, vc = d.k_cache.clone(), d.v_cache.clone()
-    used = set(np.unique(w.block_tables[w.block_tables >= 0]).tolist())
-    free = [b for b in range(w.num_blocks) if b not in used]
+    extra = 2 * full
+    pad = torch.zeros((extra,) + tuple(d.k_cache.shape[1:]), dtype=d.dt, device="cuda")
+    kc, vc = torch.cat([d.k_cache, pad]), torch.cat([d.v_cache, pad])
+    free = list(range(w.num_blocks, w.num_blocks + extra))
     bt = w.block_tables.copy()
     for s in range(1, 3):
         for j in range(full):
