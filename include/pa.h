@@ -149,6 +149,38 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t n
                          int64_t num_blocks, pa_dtype dtype, int32_t* dev_error,
                          void* stream);
 
+/*
+ * pa_decode for callers that cannot allocate device memory -- for example a
+ * plugin inside a host application that owns all device memory and forbids
+ * its plugins from calling cudaMalloc, or a latency-critical decode loop that
+ * cannot afford cudaMalloc/cudaFree (they may synchronise the whole device).
+ * The pages have no counterpart to this call; it is a deployment convenience.
+ *
+ * Same arguments and result as pa_decode, without workspace arguments: the
+ * split-K scratch is a fixed array of PA_STATIC_WORKSPACE_BYTES compiled into
+ * the library, present in each GPU's memory once the library's device code is
+ * loaded there and held until the process exits. The caller still provides
+ * every input and output buffer. The call allocates nothing.
+ *   - Sizes whose pa_decode_workspace_size(...) exceeds
+ *     PA_STATIC_WORKSPACE_BYTES return PA_ERR_WORKSPACE_TOO_SMALL and launch
+ *     nothing (use pa_decode with a caller workspace for those).
+ *   - The first call on a device looks the array's address up on that device
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture on the device.
+ *   - All calls on a device share the array. Nothing in it needs to start at
+ *     zero, but calls whose kernels overlap on the GPU race on it: order them
+ *     on one stream or with events.
+ */
+#define PA_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+pa_status pa_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int32_t block_table_stride,
+                           const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                           int32_t group_size, int32_t head_dim, int32_t block_size,
+                           int64_t num_blocks, int32_t max_context_len, float scale,
+                           int32_t partition_tokens, int32_t* dev_error, pa_dtype dtype,
+                           void* stream);
+
 /* Static description of a status code. */
 const char* pa_status_string(pa_status status);
 

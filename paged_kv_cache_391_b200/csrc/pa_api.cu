@@ -76,6 +76,10 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
+namespace pa {
+pa_status record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace pa
+
 extern "C" {
 
 const char* pa_status_string(pa_status s) {

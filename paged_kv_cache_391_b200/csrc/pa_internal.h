@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "pa.h"
+
 namespace pa {
 
 struct DecodeLaunch {
@@ -35,6 +37,9 @@ struct DecodeLaunch {
 };
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+
+// Records a CUDA error for pa_last_cuda_error() and returns PA_ERR_CUDA.
+pa_status record_cuda_error(cudaError_t e);
 
 cudaError_t launch_write_kv(const void* k, const void* v, void* k_cache, void* v_cache,
                             const int64_t* slot_mapping, int32_t num_tokens,

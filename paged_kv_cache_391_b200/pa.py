@@ -23,7 +23,8 @@ PA_DEV_ERR_TIMEOUT = 1 << 24
 
 # Every entry point include/pa.h declares.
 EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_blocks",
-           "pa_status_string", "pa_last_cuda_error")
+           "pa_status_string", "pa_last_cuda_error", "pa_decode_static")
+PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
 _lib = None
@@ -56,6 +57,9 @@ def lib() -> ctypes.CDLL:
             L.pa_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, i32,
                                     ctypes.c_float, i32, P, sz, P, ctypes.c_int, P]
             L.pa_decode.restype = ctypes.c_int
+            L.pa_decode_static.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
+                                           i32, ctypes.c_float, i32, P, ctypes.c_int, P]
+            L.pa_decode_static.restype = ctypes.c_int
             L.pa_copy_blocks.argtypes = [P, P, i32, P, i32, i32, i32, i32, i64, ctypes.c_int, P, P]
             L.pa_copy_blocks.restype = ctypes.c_int
             L.pa_status_string.argtypes = [ctypes.c_int]
@@ -152,6 +156,30 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
                          int(partition_tokens), _ptr(workspace), ws_bytes, _ptr(dev_error),
                          _dtype_code(q), _stream(stream, q.device))
     _check(st, "pa_decode")
+    return out
+
+
+def decode_static(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, *,
+                  scale: float, max_context_len: int, partition_tokens: int = 512,
+                  dev_error: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """pa_decode without a caller workspace, for callers that may not allocate
+    device memory: the split-K scratch is a fixed array inside libpa
+    (PA_STATIC_WORKSPACE_BYTES per GPU). Calls on one device must not overlap
+    on the GPU; the first call on a device should precede any stream capture."""
+    S, Hq, D = q.shape
+    NB, Hkv = k_cache.shape[:2]
+    assert out.shape == q.shape and out.dtype == q.dtype == k_cache.dtype == v_cache.dtype
+    assert k_cache.shape == v_cache.shape == (NB, Hkv, PA_BLOCK_SIZE, D)
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    if Hq % Hkv:
+        raise ValueError("num_q_heads must be a multiple of num_kv_heads")
+    st = lib().pa_decode_static(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,
+                                Hq, Hq // Hkv, D, PA_BLOCK_SIZE, NB, int(max_context_len),
+                                float(scale), int(partition_tokens), _ptr(dev_error),
+                                _dtype_code(q), _stream(stream, q.device))
+    _check(st, "pa_decode_static")
     return out
 
 
