@@ -137,7 +137,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
       num_q_heads % group_size != 0 || partition_tokens % PA_BLOCK_SIZE != 0)
     return PA_ERR_UNSUPPORTED;
   const int32_t num_kv_heads = num_q_heads / group_size;
-  if (num_seqs > 65535 || num_kv_heads > 65535 || num_blocks > (int64_t(1) << 32))
+  if (num_seqs > 65535 || num_kv_heads > 65535 || num_blocks > (int64_t(1) << 32) ||
+      (int64_t)num_seqs * num_q_heads > 0x7fffffff)
     return PA_ERR_UNSUPPORTED;
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)

@@ -12,8 +12,8 @@
 //
 // Design (B200):
 //  * One CTA per (partition, KV head, sequence); its four warps take the
-//    partition's 16-token blocks round-robin, each with a private 3-stage ring
-//    of shared-memory tiles. A tile (one block, one KV head: 16 x D values,
+//    partition's 16-token blocks round-robin, each with a private 2-stage ring
+//    of shared-memory tiles (three CTAs per SM keep ~24 tiles in flight). A tile (one block, one KV head: 16 x D values,
 //    contiguous in HBM) arrives by TMA as 64-column boxes with a 128-byte
 //    swizzle, so the ldmatrix reads below are bank-conflict free. Completion
 //    is tracked by one mbarrier per stage; every wait is bounded.
@@ -35,14 +35,25 @@
 
 namespace pa {
 
+// CTA shape: warps per CTA and shared-memory stages per warp (compile-time).
+// 4 warps x 2 stages = 64 KiB of tiles per CTA, three CTAs per SM: measured on
+// B200 to beat deeper rings with fewer resident CTAs (2 or 1 per SM), because
+// the CTAs' start-up and merge phases then overlap other CTAs' streaming.
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2
+#endif
+
 constexpr int kBlockTokens = 16;
-constexpr int kWarps = 4;
+constexpr int kWarps = PA_DECODE_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr unsigned kFull = 0xffffffffu;
 
 template <int D>
 struct DecodeSmem {
-  static constexpr int kStages = 3;
+  static constexpr int kStages = PA_DECODE_STAGES;
   static constexpr int kSubTiles = D / 64;                 // 128-byte TMA boxes per tile
   static constexpr int kTileBytes = kBlockTokens * D * 2;  // K (or V) of one block, one KV head
   static constexpr int kStageBytes = 2 * kTileBytes;
@@ -375,83 +386,163 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// Combine the partitions of one (sequence, query head): weights
-// 2^(lse_p - max lse), normalised; fixed summation order (deterministic).
+// Combine the partitions of each (sequence, query head) row:
+//   out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M),  M = max_p lse_p.
+// Two phases, so the partial loads do not wait on each other: the weights
+// first (max and sum in a fixed order), then independent weighted loads.
+// Deterministic: the summation order depends only on the partition count.
+constexpr int kReduceWarps = 8;
+constexpr int kWarpRowMaxParts = 16;  // up to this many, one warp (half-warp) per row
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kReduceWarps * 32)
     lse_reduce_kernel(T* __restrict__ out, const float* __restrict__ part_o,
                       const float* __restrict__ part_lse, const int32_t* __restrict__ context_lens,
-                      int num_q_heads, int max_context_len, int part_tokens, int max_parts) {
-  constexpr int kW = 8;
-  constexpr int kLanes = D / 4;            // float4 columns per partition row
+                      int num_rows, int num_q_heads, int max_context_len, int part_tokens,
+                      int max_parts) {
+  constexpr int kLanes = D / 4;             // float4 columns of a row = lanes per row
   constexpr int kRowsPerWarp = 32 / kLanes;
-  constexpr int kStreams = kW * kRowsPerWarp;
   using E = Elem<T>;
-  const int hq = blockIdx.x, seq = blockIdx.y;
-  int L = context_lens[seq];
-  L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
-  const int n = (L + part_tokens - 1) / part_tokens;
-  if (n <= 1) return;  // written directly by the partition kernel
-  const size_t row = (size_t)seq * num_q_heads + hq;
-  const float* lse = part_lse + row * max_parts;
-  const float4* po = reinterpret_cast<const float4*>(part_o + row * max_parts * D);
-  __shared__ float red[kW];
-  __shared__ float4 acc_s[kStreams][kLanes];
-  __shared__ float ws_s[kStreams];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-
-  float M = -INFINITY;
-  for (int p = tid; p < n; p += kW * 32) M = fmaxf(M, lse[p]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-  if (lane == 0) red[w] = M;
-  __syncthreads();
-  M = red[0];
-#pragma unroll
-  for (int i = 1; i < kW; ++i) M = fmaxf(M, red[i]);
-
-  const int stream = w * kRowsPerWarp + lane / kLanes;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row = (blockIdx.x * kReduceWarps + warp) * kRowsPerWarp + lane / kLanes;
   const int c = lane % kLanes;
+  const unsigned grp = kRowsPerWarp == 1 ? kFull : (0xffffu << (lane & ~(kLanes - 1)));
+  int n = 0;
+  if (row < num_rows) {
+    int L = context_lens[row / num_q_heads];
+    L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
+    n = (L + part_tokens - 1) / part_tokens;
+  }
+  // n is uniform within a row's lane group; rows with n <= 1 were written directly
+  if (n <= 1) return;
+  const float* lse = part_lse + (size_t)row * max_parts;
+  const float4* po = reinterpret_cast<const float4*>(part_o + (size_t)row * max_parts * D);
+
+  const float my_lse = c < n ? lse[c] : -INFINITY;
+  float M = my_lse;
+#pragma unroll
+  for (int o = kLanes / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(grp, M, o, kLanes));
+  const float my_w = (M == -INFINITY || my_lse == -INFINITY) ? 0.f : exp2f(my_lse - M);
+  float W = my_w;
+#pragma unroll
+  for (int o = kLanes / 2; o > 0; o >>= 1) W += __shfl_xor_sync(grp, W, o, kLanes);
+
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float ws = 0.f;
-  if (M != -INFINITY) {
-#pragma unroll 4
-    for (int p = stream; p < n; p += kStreams) {
-      const float wt = exp2f(lse[p] - M);
+#pragma unroll
+  for (int p = 0; p < kWarpRowMaxParts; ++p) {
+    const float wp = __shfl_sync(grp, my_w, p, kLanes);
+    if (p < n) {
       const float4 v = po[(size_t)p * kLanes + c];
-      ws += wt;
-      acc.x += wt * v.x;
-      acc.y += wt * v.y;
-      acc.z += wt * v.z;
-      acc.w += wt * v.w;
+      acc.x += wp * v.x;
+      acc.y += wp * v.y;
+      acc.z += wp * v.z;
+      acc.w += wp * v.w;
     }
   }
-  acc_s[stream][c] = acc;
-  if (c == 0) ws_s[stream] = ws;
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (W > 0.f) {
+    res.x = acc.x / W;
+    res.y = acc.y / W;
+    res.z = acc.z / W;
+    res.w = acc.w / W;
+  }
+  uint2 pk;
+  pk.x = E::pack(res.x, res.y);
+  pk.y = E::pack(res.z, res.w);
+  *reinterpret_cast<uint2*>(out + (size_t)row * D + c * 4) = pk;
+}
+
+// Rows with many partitions (long contexts): one CTA per row. Phase 1 puts
+// the weights of all partitions in shared memory; phase 2 has every warp
+// (half-warp at D = 64) stream an interleaved subset of the partials; a
+// fixed-order merge of the streams ends it.
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32)
+    lse_reduce_split_kernel(T* __restrict__ out, const float* __restrict__ part_o,
+                            const float* __restrict__ part_lse,
+                            const int32_t* __restrict__ context_lens, int num_q_heads,
+                            int max_context_len, int part_tokens, int max_parts) {
+  constexpr int kThreadsR = kReduceWarps * 32;
+  constexpr int kLanes = D / 4;
+  constexpr int kStreams = kThreadsR / kLanes;
+  using E = Elem<T>;
+  extern __shared__ float s_w[];  // [max_parts] weights
+  __shared__ float s_red[kThreadsR];
+  __shared__ float4 s_acc[kStreams][kLanes];
+  const int row = blockIdx.x;
+  int L = context_lens[row / num_q_heads];
+  L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
+  const int n = (L + part_tokens - 1) / part_tokens;
+  if (n <= 1) return;
+  const int tid = threadIdx.x;
+  const float* lse = part_lse + (size_t)row * max_parts;
+  const float4* po = reinterpret_cast<const float4*>(part_o + (size_t)row * max_parts * D);
+
+  // phase 1: M = max lse (fixed tree), weights, W = sum of weights (fixed tree)
+  float m = -INFINITY;
+  for (int p = tid; p < n; p += kThreadsR) {
+    const float l = lse[p];
+    s_w[p] = l;
+    m = fmaxf(m, l);
+  }
+  s_red[tid] = m;
+  __syncthreads();
+  for (int o = kThreadsR / 2; o > 0; o >>= 1) {
+    if (tid < o) s_red[tid] = fmaxf(s_red[tid], s_red[tid + o]);
+    __syncthreads();
+  }
+  const float M = s_red[0];
+  __syncthreads();
+  float w = 0.f;
+  for (int p = tid; p < n; p += kThreadsR) {
+    const float l = s_w[p];
+    const float e = (M == -INFINITY || l == -INFINITY) ? 0.f : exp2f(l - M);
+    s_w[p] = e;
+    w += e;
+  }
+  s_red[tid] = w;
+  __syncthreads();
+  for (int o = kThreadsR / 2; o > 0; o >>= 1) {
+    if (tid < o) s_red[tid] += s_red[tid + o];
+    __syncthreads();
+  }
+  const float W = s_red[0];
+
+  // phase 2: independent weighted loads, one stream per warp (half-warp)
+  const int stream = tid / kLanes, c = tid % kLanes;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int p = stream; p < n; p += kStreams) {
+    const float wp = s_w[p];
+    const float4 v = po[(size_t)p * kLanes + c];
+    acc.x += wp * v.x;
+    acc.y += wp * v.y;
+    acc.z += wp * v.z;
+    acc.w += wp * v.w;
+  }
+  s_acc[stream][c] = acc;
   __syncthreads();
   if (tid < kLanes) {
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    float s = 0.f;
 #pragma unroll
     for (int i = 0; i < kStreams; ++i) {
-      const float4 v = acc_s[i][tid];
+      const float4 v = s_acc[i][tid];
       a.x += v.x;
       a.y += v.y;
       a.z += v.z;
       a.w += v.w;
-      s += ws_s[i];
     }
     float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (s > 0.f) {
-      res.x = a.x / s;
-      res.y = a.y / s;
-      res.z = a.z / s;
-      res.w = a.w / s;
+    if (W > 0.f) {
+      res.x = a.x / W;
+      res.y = a.y / W;
+      res.z = a.z / W;
+      res.w = a.w / W;
     }
     uint2 pk;
     pk.x = E::pack(res.x, res.y);
     pk.y = E::pack(res.z, res.w);
-    *reinterpret_cast<uint2*>(out + row * D + tid * 4) = pk;
+    *reinterpret_cast<uint2*>(out + (size_t)row * D + tid * 4) = pk;
   }
 }
 
@@ -468,10 +559,24 @@ static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
       a.max_context_len, a.scale_log2, a.part_blocks, a.max_parts, a.dev_error);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.max_parts <= 1) return e;
-  dim3 rgrid(a.num_q_heads, a.num_seqs);
-  lse_reduce_kernel<T, D><<<rgrid, 256, 0, stream>>>(
-      static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.num_q_heads,
-      a.max_context_len, a.part_tokens, a.max_parts);
+  const int rows = a.num_seqs * a.num_q_heads;
+  if (a.max_parts > kWarpRowMaxParts) {
+    const size_t wbytes = (size_t)a.max_parts * sizeof(float);
+    if (wbytes > 48 * 1024) {
+      e = cudaFuncSetAttribute(lse_reduce_split_kernel<T, D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
+      if (e != cudaSuccess) return e;
+    }
+    lse_reduce_split_kernel<T, D><<<rows, kReduceWarps * 32, wbytes, stream>>>(
+        static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.num_q_heads,
+        a.max_context_len, a.part_tokens, a.max_parts);
+  } else {
+    const int rows_per_cta = kReduceWarps * (32 / (D / 4));
+    lse_reduce_kernel<T, D><<<(rows + rows_per_cta - 1) / rows_per_cta, kReduceWarps * 32, 0,
+                              stream>>>(static_cast<T*>(a.out), a.part_o, a.part_lse,
+                                        a.context_lens, rows, a.num_q_heads, a.max_context_len,
+                                        a.part_tokens, a.max_parts);
+  }
   return cudaGetLastError();
 }
 

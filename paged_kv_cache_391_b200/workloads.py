@@ -86,6 +86,17 @@ class DecodeWorkload:
         return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * 2 * \
             self.head_dim * self.elem_bytes
 
+    def unique_kv_bytes(self) -> int:
+        """K and V bytes of the distinct cache slots the decode reads (blocks
+        shared by several tables counted once)."""
+        used = {}
+        for s, L in enumerate(self.context_lens):
+            L = int(L)
+            for j in range(-(-L // self.block_size)):
+                p = int(self.block_tables[s, j])
+                used[p] = max(used.get(p, 0), min(self.block_size, L - j * self.block_size))
+        return sum(used.values()) * self.num_kv_heads * 2 * self.head_dim * self.elem_bytes
+
     def step_bytes(self) -> dict:
         """Algorithmic bytes per step, by operation."""
         S, Hq, D, Hkv = self.num_seqs, self.num_q_heads, self.head_dim, self.num_kv_heads

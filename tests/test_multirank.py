@@ -1,0 +1,68 @@
+"""The multi-GPU bookkeeping of bench.py on CPU: world size 2 over gloo.
+
+Each rank runs an independent workload (weak scaling); the only collectives
+are the timing reduction (max of times, sum of work). Here the ranks hand in
+different numbers and must agree on the same whole-job figures.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    from paged_kv_cache_391_b200 import workloads as W
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = bench.make_workload("gqa", 4, seed_offset=rank)
+        elapsed = 10.0 + 5.0 * rank
+        agg = bench.reduce_over_ranks(elapsed, 20.0 - rank, w.kv_bytes(), w.num_seqs, rank,
+                                      world, device=None)
+        q.put((rank, agg, w.kv_bytes(), int(w.context_lens.sum())))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_two_ranks_agree_on_whole_job_figures():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.SimpleQueue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get() for _ in range(world))
+    (r0, a0, kv0, t0), (r1, a1, kv1, t1) = res
+    assert a0 == a1                                   # every rank sees the same figures
+    assert a0["ms"] == 15.0 and a0["e2e_ms"] == 20.0  # slowest rank
+    assert a0["kv"] == kv0 + kv1 and a0["seqs"] == 8 and a0["errors"] == 1
+    assert t0 != t1                                   # ranks ran different (independent) workloads
+
+
+def test_single_rank_is_the_identity():
+    import bench
+    agg = bench.reduce_over_ranks(3.0, 4.0, 100, 7, 0, 1)
+    assert agg == {"ms": 3.0, "e2e_ms": 4.0, "kv": 100.0, "seqs": 7.0, "errors": 0}
