@@ -74,6 +74,35 @@ def make_workload(name, batch, seed_offset=0):
     return fn(seed=seed, **kw)
 
 
+KERNEL_SOURCES = ("paged_kv_cache_391_b200/csrc/pa_decode.cu",
+                  "paged_kv_cache_391_b200/csrc/pa_device.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, batch):
+    """DRAM bytes (read + write) per pa_decode call from the ncu capture
+    recorded in profiles/dram_traffic.txt for this workload, or None when
+    there is none or the kernel sources changed since it was taken."""
+    if batch is not None or not os.path.exists(TRAFFIC_FILE):
+        return None
+    want = kernel_source_hash()
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split("#")[0].split()
+            if len(parts) >= 3 and parts[0] == workload and parts[1] == want:
+                return int(parts[2])
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -196,6 +225,44 @@ def oracle_sample(w, target_s: float):
 
 # --------------------------------------------------------------------------- GPU leg
 
+class PackedInputs:
+    """A step's inputs (q, new K/V rows, slots, CoW pairs, tables, lengths)
+    packed at 256-byte aligned offsets in one buffer, so a whole step's
+    inputs cross from pinned host memory in one copy."""
+
+    def __init__(self, w, dt, pin: bool = True):
+        import torch
+        self.dt = dt
+        parts = [("q", w.q.view(np.int16)), ("new_k", w.new_k.view(np.int16)),
+                 ("new_v", w.new_v.view(np.int16)), ("slots", w.slot_mapping),
+                 ("pairs", w.copy_pairs), ("bt", w.block_tables), ("cl", w.context_lens)]
+        self.layout, off = {}, 0
+        for name, a in parts:
+            a = np.ascontiguousarray(a)
+            self.layout[name] = (off, a.dtype, a.shape, a.nbytes)
+            off += (a.nbytes + 255) // 256 * 256
+        self.nbytes = off
+        self.host = torch.empty(off, dtype=torch.uint8)
+        if pin:
+            self.host = self.host.pin_memory()
+        hv = self.host.numpy()
+        for name, a in parts:
+            o, dtype, shape, n = self.layout[name]
+            hv[o:o + n] = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+        self.payload = sum(v[3] for v in self.layout.values())
+
+    def views(self, buf):
+        """Typed tensor views of a device buffer laid out like the host one."""
+        import torch
+        tmap = {np.dtype(np.int16): torch.int16, np.dtype(np.int64): torch.int64,
+                np.dtype(np.int32): torch.int32}
+        out = {}
+        for name, (o, dtype, shape, n) in self.layout.items():
+            t = buf[o:o + n].view(tmap[np.dtype(dtype)]).view(shape)
+            out[name] = t.view(self.dt) if dtype == np.int16 else t
+        return out
+
+
 def run_gpu(args, rank, world, device):
     import torch
     from paged_kv_cache_391_b200 import pa
@@ -209,11 +276,10 @@ def run_gpu(args, rank, world, device):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dt).to(device)
 
     k_cache, v_cache = dev16(w.k_pool), dev16(w.v_pool)
-    q, new_k, new_v = dev16(w.q), dev16(w.new_k), dev16(w.new_v)
-    slots = torch.from_numpy(w.slot_mapping).to(device)
-    pairs = torch.from_numpy(w.copy_pairs).to(device)
-    bt = torch.from_numpy(w.block_tables).to(device)
-    cl = torch.from_numpy(w.context_lens).to(device)
+    packed = PackedInputs(w, dt)
+    resident = torch.empty(packed.nbytes, dtype=torch.uint8, device=device)
+    resident.copy_(packed.host)
+    inp = packed.views(resident)
     out = torch.empty(w.q.shape, dtype=dt, device=device)
     P = w.partition_tokens
     ws = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, P, device)
@@ -226,14 +292,16 @@ def run_gpu(args, rank, world, device):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def step(e_dec=None):
-        if pairs.numel():
-            pa.copy_blocks([k_cache], [v_cache], pairs, dev_error=err, stream=stream)
-        pa.write_kv(new_k, new_v, k_cache, v_cache, slots, dev_error=err, stream=stream)
+    def step(x, o, e_dec=None):
+        if x["pairs"].numel():
+            pa.copy_blocks([k_cache], [v_cache], x["pairs"], dev_error=err, stream=stream)
+        pa.write_kv(x["new_k"], x["new_v"], k_cache, v_cache, x["slots"], dev_error=err,
+                    stream=stream)
         if e_dec is not None:
             e_dec[0].record(stream)
-        pa.decode(out, q, k_cache, v_cache, bt, cl, scale=w.scale, max_context_len=max_ctx,
-                  partition_tokens=P, workspace=ws, dev_error=err, stream=stream)
+        pa.decode(o, x["q"], k_cache, v_cache, x["bt"], x["cl"], scale=w.scale,
+                  max_context_len=max_ctx, partition_tokens=P, workspace=ws, dev_error=err,
+                  stream=stream)
         if e_dec is not None:
             e_dec[1].record(stream)
 
@@ -244,7 +312,7 @@ def run_gpu(args, rank, world, device):
         torch.cuda.synchronize(device)
 
     for _ in range(args.warmup):
-        step()
+        step(inp, out)
     barrier()
     dec_events = [(ev(), ev()) for _ in range(args.steps)]
     t_start, t_end = ev(), ev()
@@ -252,46 +320,60 @@ def run_gpu(args, rank, world, device):
         barrier()
         t_start.record(stream)
         for i in range(args.steps):
-            step(dec_events[i])
+            step(inp, out, dec_events[i])
         t_end.record(stream)
         barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in dec_events]))
     errors = int(err.item())
 
-    # ---- e2e: host buffers through the public API, copies inside the timed region
+    # ---- e2e: every step uploads its packed inputs from pinned host memory
+    # and reads its output back. Two input/output slots, an upload stream and
+    # a download stream let step i+1's upload and step i's download overlap
+    # step i's kernels.
     e2e = None
     if not args.no_e2e:
-        host = {k: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16
-                                    else np.ascontiguousarray(a)).pin_memory()
-                for k, a in (("q", w.q), ("k", w.new_k), ("v", w.new_v),
-                             ("slots", w.slot_mapping), ("bt", w.block_tables),
-                             ("cl", w.context_lens))}
-        out_host = torch.empty(out.shape, dtype=dt).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = out_host.numel() * out_host.element_size()
+        up_stream, down_stream = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        dev_in = [torch.empty(packed.nbytes, dtype=torch.uint8, device=device) for _ in range(2)]
+        views = [packed.views(b) for b in dev_in]
+        outs = [torch.empty_like(out) for _ in range(2)]
+        host_out = [torch.empty(out.shape, dtype=dt).pin_memory() for _ in range(2)]
+        uploaded = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
+        downloaded = [torch.cuda.Event() for _ in range(2)]
+        started = [False, False]
 
-        def e2e_step():
-            q.view(torch.int16).copy_(host["q"], non_blocking=True)
-            new_k.view(torch.int16).copy_(host["k"], non_blocking=True)
-            new_v.view(torch.int16).copy_(host["v"], non_blocking=True)
-            slots.copy_(host["slots"], non_blocking=True)
-            bt.copy_(host["bt"], non_blocking=True)
-            cl.copy_(host["cl"], non_blocking=True)
-            step()
-            out_host.copy_(out, non_blocking=True)
+        def e2e_step(i):
+            k = i % 2
+            with torch.cuda.stream(up_stream):
+                if started[k]:
+                    up_stream.wait_event(computed[k])       # slot k's last step has read its inputs
+                dev_in[k].copy_(packed.host, non_blocking=True)
+                uploaded[k].record(up_stream)
+            stream.wait_event(uploaded[k])
+            if started[k]:
+                stream.wait_event(downloaded[k])            # outs[k] has been read back
+            step(views[k], outs[k])
+            computed[k].record(stream)
+            with torch.cuda.stream(down_stream):
+                down_stream.wait_event(computed[k])
+                host_out[k].copy_(outs[k], non_blocking=True)
+                downloaded[k].record(down_stream)
+            started[k] = True
 
-        for _ in range(args.warmup):
-            e2e_step()
+        for i in range(args.warmup):
+            e2e_step(i)
         barrier()
         a, b = ev(), ev()
         a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        up_stream.wait_event(a)                             # no upload starts before the clock
+        for i in range(args.steps):
+            e2e_step(args.warmup + i)
+        stream.wait_stream(down_stream)
         b.record(stream)
         barrier()
-        e2e_ms = a.elapsed_time(b)
-        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+        e2e = {"ms": a.elapsed_time(b), "h2d": packed.payload,
+               "d2h": host_out[0].numel() * host_out[0].element_size()}
     return w, elapsed_ms, dec_ms, errors, clocks.report(), e2e, launches_per_step
 
 
@@ -396,7 +478,10 @@ def main():
             "unit": "GB/s",
             "frac": round(dec_achieved / peak, 4),
             "algorithmic_bytes_per_launch": sb["decode"],
-            "traffic": None,
+            "traffic": recorded_traffic(args.workload, args.batch),
+            "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                            "decode_partition_kernel + lse_reduce per call "
+                            "(profiles/dram_traffic.txt; null if the kernel changed since)",
         },
         "sub_ms": {"decode": round(dec_ms, 5),
                    "write_kv_and_copies": round(elapsed_ms / K - dec_ms, 5)},
