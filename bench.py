@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--workload", default="mha", choices=list(WORKLOAD_TEXT))
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling only)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="step", choices=["step", "swap"],
+                    help="step: the decode step (default); swap: preemption swap-out/in")
     ap.add_argument("--partition-tokens", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -406,6 +408,70 @@ def reduce_over_ranks(elapsed_ms, e2e_ms, kv_bytes, seqs, errors, world, device=
             "errors": int(s[2])}
 
 
+def run_swap(args, device):
+    """Preemption of half the batch: swap its blocks (K and V, one layer) to a
+    pinned host pool and back, timed per direction with CUDA events, next to
+    a same-size contiguous pinned copy by the copy engine (the host link's
+    ceiling, measured in the same run)."""
+    import torch
+    from paged_kv_cache_391_b200 import pa
+    w = make_workload(args.workload, args.batch)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    kc = torch.from_numpy(w.k_pool.view(np.int16)).view(dt).to(device)
+    vc = torch.from_numpy(w.v_pool.view(np.int16)).view(dt).to(device)
+    ids = set()
+    for s in range(w.num_seqs // 2):
+        n = -(-int(w.context_lens[s]) // 16)
+        ids.update(int(b) for b in w.block_tables[s, :n])
+    ids = sorted(ids)
+    n = len(ids)
+    shape = (n,) + tuple(kc.shape[1:])
+    hk = torch.empty(shape, dtype=dt).pin_memory()
+    hv = torch.empty(shape, dtype=dt).pin_memory()
+    out_map = torch.tensor([[b, i] for i, b in enumerate(ids)], dtype=torch.int64, device=device)
+    in_map = torch.tensor([[i, b] for i, b in enumerate(ids)], dtype=torch.int64, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    nbytes = 2 * hk.numel() * hk.element_size()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed(f):
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for _ in range(args.steps):
+            f()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    t_out = timed(lambda: pa.swap_blocks([kc], [vc], [hk], [hv], out_map, dev_error=err))
+    t_in = timed(lambda: pa.swap_blocks([hk], [hv], [kc], [vc], in_map, dev_error=err))
+    dk = torch.empty(shape, dtype=dt, device=device)
+    dv = torch.empty(shape, dtype=dt, device=device)
+    t_ce_out = timed(lambda: (hk.copy_(dk, non_blocking=True), hv.copy_(dv, non_blocking=True)))
+    t_ce_in = timed(lambda: (dk.copy_(hk, non_blocking=True), dv.copy_(hv, non_blocking=True)))
+    g = lambda ms: nbytes / (ms / 1e3) / 1e9  # noqa: E731
+    line = {
+        "metric": "KV block swap GB/s (device <-> pinned host), preemption of half the batch",
+        "value": round(2 * nbytes / ((t_out + t_in) / 1e3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "blocks": n, "bytes_per_direction": nbytes,
+                   "layers": 1},
+        "swap_out_GBs": round(g(t_out), 2), "swap_in_GBs": round(g(t_in), 2),
+        "roofline": {"bound": "host link", "peak_out_GBs": round(g(t_ce_out), 2),
+                     "peak_in_GBs": round(g(t_ce_in), 2),
+                     "peak_source": "contiguous pinned copy of the same bytes by the copy engine, "
+                                    "same run",
+                     "frac_out": round(t_ce_out / t_out, 4), "frac_in": round(t_ce_in / t_in, 4)},
+        "gpu_launches": 2 * args.steps, "device_errors": int(err.item()),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -421,6 +487,8 @@ def main():
         return 1
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.op == "swap":
+        return run_swap(args, device) if rank == 0 else 0
     if world > 1:
         import datetime
         import torch.distributed as dist

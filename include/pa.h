@@ -150,6 +150,29 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t n
                          void* stream);
 
 /*
+ * Swap whole blocks between two pools for preemption: a request's blocks go
+ * from GPU memory to CPU RAM and come back later ("PagedAttention",
+ * "Managing Virtual Memory (Block Manager)": inactive KV blocks are swapped
+ * to CPU RAM and brought back when needed; "The Memory Wall ...", "The Block
+ * Manager": preempt a request, save its state, resume later). For each pair p
+ * and layer l: dst_k[l][mapping[2p+1]] = src_k[l][mapping[2p]], same for V.
+ *   src_k, src_v, dst_k, dst_v  HOST arrays of num_layers pool pointers; each
+ *                   pool is device memory or pinned / registered host memory
+ *                   ([num_blocks][num_kv_heads][16][head_dim], 16-byte aligned)
+ *   block_mapping   int64 [num_pairs][2] (src, dst), device or pinned host
+ *   src_num_blocks, dst_num_blocks  pool sizes in blocks (pairs outside them
+ *                   are skipped and counted in dev_error)
+ * Pageable host memory is refused with PA_ERR_INVALID_ARG before any launch.
+ * The copy runs as one kernel on `stream` (host pools cross the host link).
+ * A dst that repeats is undefined.
+ */
+pa_status pa_swap_blocks(void* const* src_k, void* const* src_v, void* const* dst_k,
+                         void* const* dst_v, int32_t num_layers, const int64_t* block_mapping,
+                         int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t block_size, int64_t src_num_blocks, int64_t dst_num_blocks,
+                         pa_dtype dtype, int32_t* dev_error, void* stream);
+
+/*
  * pa_decode for callers that cannot allocate device memory -- for example a
  * plugin inside a host application that owns all device memory and forbids
  * its plugins from calling cudaMalloc, or a latency-critical decode loop that

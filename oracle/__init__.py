@@ -14,6 +14,8 @@ What each function follows, by page and section:
 * ``copy_blocks`` -- same page, "Copy-on-Write"; and "PagedAttention"
   (ai-system-design-guide), "KV Cache Sharing (Copy-on-Write)": a shared block
   is copied when one sequence diverges, the shared original stays unchanged.
+* ``swap_blocks`` -- "PagedAttention", "Managing Virtual Memory (Block
+  Manager)": blocks move between GPU memory and CPU RAM and back.
 * ``decode`` -- same first page, "PagedAttention: Decoupling Logical Context
   from Contiguous GPU Memory" (Figure 2), and "The Memory Wall ...", "How it
   Works Under the Hood" and "Show Me The Code": the kernel walks the block
@@ -65,6 +67,8 @@ def _load():
             lib.oracle_write_kv.restype = i64
             lib.oracle_copy_blocks.argtypes = [P, P, i32, P, i32, i32, i32, i32]
             lib.oracle_copy_blocks.restype = None
+            lib.oracle_swap_blocks.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32]
+            lib.oracle_swap_blocks.restype = None
             lib.oracle_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                           ctypes.c_double, ctypes.c_int, P, i64, ctypes.c_int]
             lib.oracle_decode.restype = ctypes.c_int
@@ -121,6 +125,18 @@ def copy_blocks(k_caches, v_caches, block_mapping, block_size: int = 16) -> None
     _, H, bs, D = k_caches[0].shape
     _load().oracle_copy_blocks(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
                                L, _ptr(block_mapping), block_mapping.shape[0], H, D, bs)
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, block_size: int = 16) -> None:
+    """Copy whole blocks ``src -> dst`` from per-layer source pools into
+    per-layer destination pools (lists of ``[NB, H_kv, 16, D]`` uint16 arrays;
+    the two sides may have different block counts), in place."""
+    block_mapping = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+    L = len(src_k)
+    arrs = [(ctypes.c_void_p * L)(*[_ptr(c) for c in side]) for side in (src_k, src_v, dst_k, dst_v)]
+    _, H, bs, D = src_k[0].shape
+    _load().oracle_swap_blocks(*[ctypes.cast(a, ctypes.c_void_p) for a in arrs], L,
+                               _ptr(block_mapping), block_mapping.shape[0], H, D, bs)
 
 
 def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype,

@@ -137,6 +137,28 @@ void oracle_copy_blocks(uint16_t** k_caches, uint16_t** v_caches, int32_t num_la
   }
 }
 
+/*
+ * Swap blocks between two pools (preemption moves a request's blocks from GPU
+ * memory to CPU RAM and back: "PagedAttention", "Managing Virtual Memory
+ * (Block Manager)"): for every (src, dst) pair and every layer, block src of
+ * the source pool is copied whole to block dst of the destination pool.
+ */
+void oracle_swap_blocks(uint16_t** src_k, uint16_t** src_v, uint16_t** dst_k, uint16_t** dst_v,
+                        int32_t num_layers, const int64_t* block_mapping, int32_t num_pairs,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t block_size) {
+  size_t block_elems = (size_t)num_kv_heads * block_size * head_dim;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    for (int32_t p = 0; p < num_pairs; ++p) {
+      int64_t src = block_mapping[2 * p];
+      int64_t dst = block_mapping[2 * p + 1];
+      memcpy(dst_k[l] + dst * block_elems, src_k[l] + src * block_elems,
+             block_elems * sizeof(uint16_t));
+      memcpy(dst_v[l] + dst * block_elems, src_v[l] + src * block_elems,
+             block_elems * sizeof(uint16_t));
+    }
+  }
+}
+
 typedef struct {
   const uint16_t* q;
   const uint16_t* k_cache;

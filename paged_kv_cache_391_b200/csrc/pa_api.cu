@@ -78,6 +78,28 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 namespace pa {
 pa_status record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
+pa_status device_view(const void* p, void** dev_ptr) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, p);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // do not leave this error for a later call to report
+    return PA_ERR_INVALID_ARG;
+  }
+  switch (attr.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+      *dev_ptr = const_cast<void*>(p);
+      return PA_OK;
+    case cudaMemoryTypeHost:
+      if (!attr.devicePointer) return PA_ERR_INVALID_ARG;
+      *dev_ptr = attr.devicePointer;
+      return PA_OK;
+    default:
+      return PA_ERR_INVALID_ARG;  // pageable host memory: not reachable from kernels
+  }
+}
 }  // namespace pa
 
 extern "C" {
@@ -209,9 +231,60 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t n
     if (!k_caches[l] || !v_caches[l] || !aligned(k_caches[l], 16) || !aligned(v_caches[l], 16))
       return PA_ERR_INVALID_ARG;
   const int64_t block_bytes = (int64_t)num_kv_heads * PA_BLOCK_SIZE * head_dim * 2;
-  cudaError_t e = pa::launch_copy_blocks(k_caches, v_caches, num_layers, block_mapping, num_pairs,
-                                         block_bytes, num_blocks, dev_error,
-                                         static_cast<cudaStream_t>(stream));
+  cudaError_t e = pa::launch_block_copy(k_caches, v_caches, k_caches, v_caches, num_layers,
+                                        block_mapping, num_pairs, block_bytes, num_blocks,
+                                        num_blocks, dev_error, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+pa_status pa_swap_blocks(void* const* src_k, void* const* src_v, void* const* dst_k,
+                         void* const* dst_v, int32_t num_layers, const int64_t* block_mapping,
+                         int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t block_size, int64_t src_num_blocks, int64_t dst_num_blocks,
+                         pa_dtype dtype, int32_t* dev_error, void* stream) {
+  if (num_layers < 1 || num_pairs < 0 || num_kv_heads < 1 || src_num_blocks < 1 ||
+      dst_num_blocks < 1 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_layers > PA_MAX_LAYERS || block_size != PA_BLOCK_SIZE || head_dim < 8 ||
+      head_dim % 8)
+    return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!src_k || !src_v || !dst_k || !dst_v || !block_mapping || !aligned(block_mapping, 8) ||
+      (dev_error && !aligned(dev_error, 4)))
+    return PA_ERR_INVALID_ARG;
+  // Every pool, the mapping and the error counter must be reachable from the
+  // device: device memory, managed memory, or pinned / registered host
+  // memory (translated to its device address). Pageable host memory is
+  // refused here instead of faulting in the kernel.
+  void* dk[PA_MAX_LAYERS];
+  void* dv[PA_MAX_LAYERS];
+  void* sk[PA_MAX_LAYERS];
+  void* sv[PA_MAX_LAYERS];
+  void* const* in[4] = {src_k, src_v, dst_k, dst_v};
+  void** outp[4] = {sk, sv, dk, dv};
+  for (int a = 0; a < 4; ++a) {
+    for (int l = 0; l < num_layers; ++l) {
+      void* dp = nullptr;
+      pa_status st = pa::device_view(in[a][l], &dp);
+      if (st != PA_OK) return st;
+      if (!aligned(dp, 16)) return PA_ERR_INVALID_ARG;
+      outp[a][l] = dp;
+    }
+  }
+  void* map_dp = nullptr;
+  pa_status st = pa::device_view(block_mapping, &map_dp);
+  if (st != PA_OK) return st;
+  void* err_dp = nullptr;
+  if (dev_error) {
+    st = pa::device_view(dev_error, &err_dp);
+    if (st != PA_OK) return st;
+  }
+  const int64_t block_bytes = (int64_t)num_kv_heads * PA_BLOCK_SIZE * head_dim * 2;
+  cudaError_t e = pa::launch_block_copy(sk, sv, dk, dv, num_layers,
+                                        static_cast<const int64_t*>(map_dp), num_pairs,
+                                        block_bytes, src_num_blocks, dst_num_blocks,
+                                        static_cast<int32_t*>(err_dp),
+                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 

@@ -5,11 +5,15 @@
 //    ("Optimizing LLM Inference: From PagedAttention to AI Infra",
 //    "Understanding KV Cache ..."). One CTA per token; each thread moves
 //    16-byte vectors, so a row of D = 128 bf16 values is 16 coalesced vectors.
-//  * copy_blocks: the copy-on-write fork of a shared block (same page,
-//    "Copy-on-Write"; "PagedAttention", "KV Cache Sharing (Copy-on-Write)"):
-//    the whole physical block -- every KV head, every slot -- of K and of V,
-//    in every layer. Blocks are contiguous in HBM, so this is a plain
-//    16-byte-vector copy with several vectors in flight per thread.
+//  * block copies: the copy-on-write fork of a shared block (same page,
+//    "Copy-on-Write"; "PagedAttention", "KV Cache Sharing (Copy-on-Write)")
+//    and the swap of blocks between GPU memory and CPU RAM for preemption
+//    ("PagedAttention", "Managing Virtual Memory (Block Manager)"; "The
+//    Memory Wall ...", "The Block Manager"): the whole physical block --
+//    every KV head, every slot -- of K and of V, in every layer. Blocks are
+//    contiguous, so this is a plain 16-byte-vector copy with several vectors
+//    in flight per thread; a pinned host pool is read or written in place
+//    over the host link.
 #include "pa.h"
 #include "pa_internal.h"
 
@@ -40,28 +44,35 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-struct LayerPtrs {
-  uint4* k[PA_MAX_LAYERS];
-  uint4* v[PA_MAX_LAYERS];
+// Per-layer source and destination pools of a block copy. For copy-on-write
+// both sides are the same device pool; for a swap one side is a pinned host
+// pool reached through unified addressing.
+struct PoolPtrs {
+  const uint4* src_k[PA_MAX_LAYERS];
+  const uint4* src_v[PA_MAX_LAYERS];
+  uint4* dst_k[PA_MAX_LAYERS];
+  uint4* dst_v[PA_MAX_LAYERS];
 };
 
 constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;
 
+// One CTA per (pair, layer, K or V): copies one whole block, 16-byte vectors,
+// kCopyUnroll of them in flight per thread.
 __global__ void __launch_bounds__(kCopyThreads)
-    copy_blocks_kernel(const __grid_constant__ LayerPtrs ptrs,
-                       const int64_t* __restrict__ block_mapping, int64_t vec_per_block,
-                       int64_t num_blocks, int32_t* __restrict__ dev_error) {
+    block_copy_kernel(const __grid_constant__ PoolPtrs ptrs,
+                      const int64_t* __restrict__ block_mapping, int64_t vec_per_block,
+                      int64_t src_num_blocks, int64_t dst_num_blocks,
+                      int32_t* __restrict__ dev_error) {
   const int pair = blockIdx.x, layer = blockIdx.y;
   const bool is_v = blockIdx.z != 0;
   const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+  if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
     if (threadIdx.x == 0 && layer == 0 && !is_v && dev_error) atomicAdd(dev_error, 1);
     return;
   }
-  uint4* base = is_v ? ptrs.v[layer] : ptrs.k[layer];
-  const uint4* s = base + src * vec_per_block;
-  uint4* d = base + dst * vec_per_block;
+  const uint4* s = (is_v ? ptrs.src_v[layer] : ptrs.src_k[layer]) + src * vec_per_block;
+  uint4* d = (is_v ? ptrs.dst_v[layer] : ptrs.dst_k[layer]) + dst * vec_per_block;
   int64_t i = threadIdx.x;
   for (; i + (kCopyUnroll - 1) * kCopyThreads < vec_per_block; i += kCopyUnroll * kCopyThreads) {
     uint4 r[kCopyUnroll];
@@ -88,18 +99,22 @@ cudaError_t launch_write_kv(const void* k, const void* v, void* k_cache, void* v
   return cudaGetLastError();
 }
 
-cudaError_t launch_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_layers,
-                               const int64_t* block_mapping, int32_t num_pairs,
-                               int64_t block_bytes, int64_t num_blocks, int32_t* dev_error,
-                               cudaStream_t stream) {
-  LayerPtrs ptrs;
+cudaError_t launch_block_copy(void* const* src_k, void* const* src_v, void* const* dst_k,
+                              void* const* dst_v, int32_t num_layers,
+                              const int64_t* block_mapping, int32_t num_pairs,
+                              int64_t block_bytes, int64_t src_num_blocks,
+                              int64_t dst_num_blocks, int32_t* dev_error, cudaStream_t stream) {
+  PoolPtrs ptrs;
   for (int l = 0; l < PA_MAX_LAYERS; ++l) {
-    ptrs.k[l] = l < num_layers ? static_cast<uint4*>(k_caches[l]) : nullptr;
-    ptrs.v[l] = l < num_layers ? static_cast<uint4*>(v_caches[l]) : nullptr;
+    const bool in = l < num_layers;
+    ptrs.src_k[l] = in ? static_cast<const uint4*>(src_k[l]) : nullptr;
+    ptrs.src_v[l] = in ? static_cast<const uint4*>(src_v[l]) : nullptr;
+    ptrs.dst_k[l] = in ? static_cast<uint4*>(dst_k[l]) : nullptr;
+    ptrs.dst_v[l] = in ? static_cast<uint4*>(dst_v[l]) : nullptr;
   }
   dim3 grid(num_pairs, num_layers, 2);
-  copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(ptrs, block_mapping, block_bytes / 16,
-                                                        num_blocks, dev_error);
+  block_copy_kernel<<<grid, kCopyThreads, 0, stream>>>(ptrs, block_mapping, block_bytes / 16,
+                                                       src_num_blocks, dst_num_blocks, dev_error);
   return cudaGetLastError();
 }
 

@@ -41,14 +41,20 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // Records a CUDA error for pa_last_cuda_error() and returns PA_ERR_CUDA.
 pa_status record_cuda_error(cudaError_t e);
 
+// The address a kernel uses for p: device and managed memory as is, pinned or
+// registered host memory through its mapped device address. Anything else
+// (pageable host memory, an unknown pointer) is PA_ERR_INVALID_ARG.
+pa_status device_view(const void* p, void** dev_ptr);
+
 cudaError_t launch_write_kv(const void* k, const void* v, void* k_cache, void* v_cache,
                             const int64_t* slot_mapping, int32_t num_tokens,
                             int32_t num_kv_heads, int32_t head_dim, int64_t num_blocks,
                             int32_t* dev_error, cudaStream_t stream);
 
-cudaError_t launch_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_layers,
-                               const int64_t* block_mapping, int32_t num_pairs,
-                               int64_t block_bytes, int64_t num_blocks, int32_t* dev_error,
-                               cudaStream_t stream);
+cudaError_t launch_block_copy(void* const* src_k, void* const* src_v, void* const* dst_k,
+                              void* const* dst_v, int32_t num_layers,
+                              const int64_t* block_mapping, int32_t num_pairs,
+                              int64_t block_bytes, int64_t src_num_blocks,
+                              int64_t dst_num_blocks, int32_t* dev_error, cudaStream_t stream);
 
 }  // namespace pa

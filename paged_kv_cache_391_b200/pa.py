@@ -23,7 +23,7 @@ PA_DEV_ERR_TIMEOUT = 1 << 24
 
 # Every entry point include/pa.h declares.
 EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_blocks",
-           "pa_status_string", "pa_last_cuda_error", "pa_decode_static")
+           "pa_status_string", "pa_last_cuda_error", "pa_decode_static", "pa_swap_blocks")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
             L.pa_decode_static.restype = ctypes.c_int
             L.pa_copy_blocks.argtypes = [P, P, i32, P, i32, i32, i32, i32, i64, ctypes.c_int, P, P]
             L.pa_copy_blocks.restype = ctypes.c_int
+            L.pa_swap_blocks.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i64, i64,
+                                         ctypes.c_int, P, P]
+            L.pa_swap_blocks.restype = ctypes.c_int
             L.pa_status_string.argtypes = [ctypes.c_int]
             L.pa_status_string.restype = ctypes.c_char_p
             L.pa_last_cuda_error.argtypes = []
@@ -199,3 +202,24 @@ def copy_blocks(k_caches, v_caches, block_mapping: torch.Tensor, *,
                               _dtype_code(k_caches[0]), _ptr(dev_error),
                               _stream(stream, k_caches[0].device))
     _check(st, "pa_copy_blocks")
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping: torch.Tensor, *,
+                dev_error: torch.Tensor | None = None, stream=None) -> None:
+    """Copy whole blocks ``src -> dst`` between two pools, layer by layer
+    (lists of ``[NB, H_kv, 16, D]`` tensors). Each pool lives in device memory
+    or in pinned host memory (``tensor.pin_memory()``); ``block_mapping`` is
+    an int64 ``[n, 2]`` tensor on the device or in pinned host memory."""
+    L = len(src_k)
+    assert L >= 1 and len(src_v) == len(dst_k) == len(dst_v) == L
+    _, H, bs, D = src_k[0].shape
+    assert dst_k[0].shape[1:] == src_k[0].shape[1:]
+    assert block_mapping.dtype == torch.int64
+    n = block_mapping.numel() // 2
+    arrs = [(ctypes.c_void_p * L)(*[_ptr(t) for t in side]) for side in (src_k, src_v, dst_k, dst_v)]
+    dev = src_k[0].device if src_k[0].is_cuda else dst_k[0].device
+    st = lib().pa_swap_blocks(*[ctypes.cast(a, ctypes.c_void_p) for a in arrs], L,
+                              _ptr(block_mapping), n, H, D, bs, src_k[0].shape[0],
+                              dst_k[0].shape[0], _dtype_code(src_k[0]), _ptr(dev_error),
+                              _stream(stream, dev))
+    _check(st, "pa_swap_blocks")

@@ -118,3 +118,19 @@ def test_missing_library_is_an_error(monkeypatch, tmp_path):
     monkeypatch.setattr(pa, "LIB_PATH", str(tmp_path / "libpa.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         pa.lib()
+
+
+def test_swap_blocks_rejects_on_the_host(L):
+    f = L.pa_swap_blocks
+    arr = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    P = ctypes.cast(arr, ctypes.c_void_p)
+    args = lambda **k: [k.get("sk", P), P, P, P, k.get("nl", 1), FAKE, k.get("n", 3), 8, 128,
+                        k.get("bs", 16), 10, 10, k.get("dt", 1), None, None]
+    assert f(*args(nl=0)) == pa.PA_ERR_INVALID_ARG
+    assert f(*args(nl=pa.PA_MAX_LAYERS + 1)) == pa.PA_ERR_UNSUPPORTED
+    assert f(*args(bs=8)) == pa.PA_ERR_UNSUPPORTED
+    assert f(*args(dt=5)) == pa.PA_ERR_INVALID_ARG
+    assert f(*args(sk=None)) == pa.PA_ERR_INVALID_ARG
+    assert f(*args(n=0)) == pa.PA_OK
+    # an address no allocation owns is refused before any launch
+    assert f(*args()) == pa.PA_ERR_INVALID_ARG

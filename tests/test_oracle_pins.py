@@ -393,3 +393,31 @@ def test_rows_subset_matches_full():
     sub = oracle.decode(w.q[:4], w.k_pool, w.v_pool, w.block_tables[:4], w.context_lens[:4] - 1,
                         w.scale, w.dtype, rows=rows)
     assert np.array_equal(sub, full.reshape(-1, 64)[rows])
+
+
+def test_swap_blocks_between_pools_of_different_sizes():
+    """Swap out (device-sized pool -> small host pool) and back in to other
+    block ids: the moved blocks are byte-identical, nothing else changes."""
+    rng = np.random.default_rng(14)
+    H, D, nl = 2, 64, 2
+    dev_k = [_bits(rng, (12, H, 16, D), "bf16") for _ in range(nl)]
+    dev_v = [_bits(rng, (12, H, 16, D), "bf16") for _ in range(nl)]
+    host_k = [np.zeros((4, H, 16, D), np.uint16) for _ in range(nl)]
+    host_v = [np.zeros((4, H, 16, D), np.uint16) for _ in range(nl)]
+    orig = [k.copy() for k in dev_k]
+    out_pairs = np.array([[3, 0], [9, 1], [4, 2]], np.int64)
+    oracle.swap_blocks(dev_k, dev_v, host_k, host_v, out_pairs)
+    for l in range(nl):
+        for s, d in out_pairs:
+            assert np.array_equal(host_k[l][d], dev_k[l][s])
+            assert np.array_equal(host_v[l][d], dev_v[l][s])
+        assert not host_k[l][3].any()
+        assert np.array_equal(dev_k[l], orig[l])          # the source is only read
+    in_pairs = np.array([[0, 11], [1, 0], [2, 5]], np.int64)
+    oracle.swap_blocks(host_k, host_v, dev_k, dev_v, in_pairs)
+    for l in range(nl):
+        assert np.array_equal(dev_k[l][11], orig[l][3])
+        assert np.array_equal(dev_k[l][0], orig[l][9])
+        assert np.array_equal(dev_k[l][5], orig[l][4])
+        untouched = [b for b in range(12) if b not in (11, 0, 5)]
+        assert np.array_equal(dev_k[l][untouched], orig[l][untouched])
