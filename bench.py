@@ -55,8 +55,9 @@ def parse():
     ap.add_argument("--workload", default="mha", choices=list(WORKLOAD_TEXT))
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling only)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="step", choices=["step", "swap"],
-                    help="step: the decode step (default); swap: preemption swap-out/in")
+    ap.add_argument("--op", default="step", choices=["step", "swap", "blockmgr"],
+                    help="step: the decode step (default); swap: preemption swap-out/in; "
+                         "blockmgr: host block-manager throughput (no GPU)")
     ap.add_argument("--partition-tokens", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -472,6 +473,53 @@ def run_swap(args, device):
     return 0
 
 
+def run_blockmgr(args):
+    """Host time of the block manager's per-step work for a GQA-sized batch:
+    256 prompts (lognormal lengths, median 1024), each forked into 4 samples
+    (1024 sequences), then `steps` decode steps of append_slots (copy-on-write
+    on the first one) + block_tables. The plain-Python model of the same rules
+    is timed beside it as the baseline."""
+    from oracle.block_manager import BlockManagerModel
+    from paged_kv_cache_391_b200 import pa
+    rng = np.random.default_rng(7)
+    lens = np.clip(np.round(np.exp(np.log(1024.0) + rng.standard_normal(256))), 16, 8192)
+    ids = list(range(1024))
+    pool = int(sum(-(-int(L) // 16) for L in lens) + 1024 * (args.steps // 16 + 2) + 1024)
+    stride = int(-(-(lens.max() + args.steps) // 16)) + 1
+
+    def drive(m, steps):
+        for i, L in enumerate(lens):
+            m.add_sequence(4 * i, int(L))
+            for c in (1, 2, 3):
+                m.fork(4 * i, 4 * i + c)
+        t0 = time.perf_counter()
+        cow = 0
+        for _ in range(steps):
+            _, c = m.append_slots(ids)
+            cow += len(c)
+            m.block_tables(ids, stride)
+        return (time.perf_counter() - t0) / steps, cow
+
+    native_s, cow = drive(pa.BlockManager(pool), args.steps)
+    model_steps = max(1, min(args.steps, 20))
+    model_s, _ = drive(BlockManagerModel(pool), model_steps)
+    line = {
+        "metric": "block-manager host time per decode step (append_slots + block_tables)",
+        "value": round(native_s * 1e6, 2), "unit": "us/step", "higher_is_better": False,
+        "steps": args.steps, "data": "synthetic",
+        "config": {"sequences": len(ids), "prompts": 256, "samples_per_prompt": 4,
+                   "prompt_lens": "lognormal(median 1024, sigma 1) clipped [16,8192]",
+                   "pool_blocks": pool, "table_stride": stride},
+        "cow_copies": cow,
+        "seq_steps_per_s": round(len(ids) / native_s, 1),
+        "cpu_baseline": {"value": round(model_s * 1e6, 2), "unit": "us/step",
+                         "kind": "plain-Python model of the same rules (oracle/block_manager.py)",
+                         "steps": model_steps, "cores": 1},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -480,6 +528,8 @@ def main():
 
     if args.impl == "reference":
         return main_reference(args, rank, world)
+    if args.op == "blockmgr":
+        return run_blockmgr(args) if rank == 0 else 0
 
     import torch
     if not torch.cuda.is_available():

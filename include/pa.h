@@ -71,7 +71,8 @@ typedef enum {
   PA_ERR_INVALID_ARG = 1,
   PA_ERR_UNSUPPORTED = 2,
   PA_ERR_WORKSPACE_TOO_SMALL = 3,
-  PA_ERR_CUDA = 4
+  PA_ERR_CUDA = 4,
+  PA_ERR_OUT_OF_BLOCKS = 5 /* block manager: not enough free blocks; nothing changed */
 } pa_status;
 
 typedef enum { PA_DTYPE_F16 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
@@ -203,6 +204,78 @@ pa_status pa_decode_static(void* out, const void* q, const void* k_cache, const 
                            int64_t num_blocks, int32_t max_context_len, float scale,
                            int32_t partition_tokens, int32_t* dev_error, pa_dtype dtype,
                            void* stream);
+
+/*
+ * Host block manager: the allocator that decides which physical block every
+ * token goes to and when a copy-on-write copy is due ("Optimizing LLM
+ * Inference ...", "On-Demand Allocation" and "Copy-on-Write"; "PagedAttention",
+ * "KV Cache Sharing (Copy-on-Write)"; "PagedAttention in Action ...", "Fixed
+ * Block Size, Mitigating External Fragmentation"; "The Memory Wall ...", "The
+ * Block Manager"). Host memory only; it produces the slot_mapping, the
+ * copy-on-write block_mapping, the block tables and the context lengths that
+ * pa_write_kv, pa_copy_blocks and pa_decode consume.
+ *
+ * Rules: a sequence holds ceil(tokens / 16) blocks; a fork shares all of its
+ * parent's blocks (reference count + 1 each); appending a token takes a new
+ * block when the last one is full, and copies the last block first when other
+ * sequences still hold it (the copy pair is reported; the last holder writes
+ * in place); freeing drops one reference per block and returns unreferenced
+ * blocks to the pool. Free blocks are handed out last-freed first, and
+ * initially in increasing id order. Every call either succeeds completely or
+ * changes nothing. A manager is not thread-safe.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+typedef struct {
+  int64_t num_blocks;     /* pool size */
+  int64_t free_blocks;
+  int64_t used_blocks;    /* num_blocks - free_blocks */
+  int64_t shared_blocks;  /* blocks held by more than one sequence */
+  int64_t sequences;
+  int64_t tokens;         /* sum of the sequences' token counts */
+  int64_t logical_blocks; /* sum of the sequences' table lengths */
+} pa_bm_stats;
+
+/* A manager of num_blocks blocks of block_size (must be 16) tokens; NULL on
+ * bad arguments or no memory. Release with pa_bm_destroy. */
+pa_block_manager* pa_bm_create(int64_t num_blocks, int32_t block_size);
+void pa_bm_destroy(pa_block_manager* bm);
+int64_t pa_bm_num_free_blocks(const pa_block_manager* bm);
+
+/* A new sequence whose first num_tokens tokens (a prompt) take
+ * ceil(num_tokens / 16) fresh blocks. PA_ERR_INVALID_ARG if seq_id exists. */
+pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, int64_t num_tokens);
+
+/* child_id shares every block of parent_id (parallel samples, beams, a shared
+ * system prompt). */
+pa_status pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id);
+
+/* Drop the sequence; blocks no other sequence holds return to the pool. */
+pa_status pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id);
+
+/* slots[t] = cache slot of logical position start + t of seq_id, for
+ * writing a prompt's K/V with pa_write_kv (positions must be < its length). */
+pa_status pa_bm_slots(const pa_block_manager* bm, int64_t seq_id, int64_t start, int64_t count,
+                      int64_t* slots);
+
+/* One decode step: reserve the slot of the next token of each of num_seqs
+ * distinct sequences (slot_mapping[i], host int64). Copy-on-write pairs
+ * (src, dst) go to cow_pairs (host int64, room for num_seqs pairs), their
+ * count to *num_cow; issue pa_copy_blocks with them before pa_write_kv.
+ * PA_ERR_OUT_OF_BLOCKS (nothing changed) when the pool cannot cover it. */
+pa_status pa_bm_append_slots(pa_block_manager* bm, const int64_t* seq_ids, int32_t num_seqs,
+                             int64_t* slot_mapping, int64_t* cow_pairs, int32_t* num_cow);
+
+/* Decode inputs for num_seqs sequences: block_tables [num_seqs][stride]
+ * (entries past each table = -1) and context_lens, both host int32. */
+pa_status pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids,
+                             int32_t num_seqs, int32_t* block_tables, int32_t stride,
+                             int32_t* context_lens);
+
+pa_status pa_bm_get_stats(const pa_block_manager* bm, pa_bm_stats* out);
+
+/* Reference count of one physical block (-1 for a bad id). */
+int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
 
 /* Static description of a status code. */
 const char* pa_status_string(pa_status status);

@@ -111,6 +111,7 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_UNSUPPORTED: return "unsupported shape or type";
     case PA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_OUT_OF_BLOCKS: return "out of KV cache blocks";
   }
   return "unknown status";
 }

@@ -15,7 +15,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpa.so")
 
-PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA = range(5)
+(PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA,
+ PA_ERR_OUT_OF_BLOCKS) = range(6)
 PA_DTYPE_F16, PA_DTYPE_BF16 = 0, 1
 PA_BLOCK_SIZE = 16
 PA_MAX_LAYERS = 256
@@ -23,7 +24,10 @@ PA_DEV_ERR_TIMEOUT = 1 << 24
 
 # Every entry point include/pa.h declares.
 EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_blocks",
-           "pa_status_string", "pa_last_cuda_error", "pa_decode_static", "pa_swap_blocks")
+           "pa_status_string", "pa_last_cuda_error", "pa_decode_static", "pa_swap_blocks",
+           "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence",
+           "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots", "pa_bm_append_slots",
+           "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -65,6 +69,24 @@ def lib() -> ctypes.CDLL:
             L.pa_swap_blocks.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i64, i64,
                                          ctypes.c_int, P, P]
             L.pa_swap_blocks.restype = ctypes.c_int
+            L.pa_bm_create.argtypes = [i64, i32]
+            L.pa_bm_create.restype = P
+            L.pa_bm_destroy.argtypes = [P]
+            L.pa_bm_destroy.restype = None
+            L.pa_bm_num_free_blocks.argtypes = [P]
+            L.pa_bm_num_free_blocks.restype = i64
+            L.pa_bm_add_sequence.argtypes = [P, i64, i64]
+            L.pa_bm_fork.argtypes = [P, i64, i64]
+            L.pa_bm_free_sequence.argtypes = [P, i64]
+            L.pa_bm_slots.argtypes = [P, i64, i64, i64, P]
+            L.pa_bm_append_slots.argtypes = [P, P, i32, P, P, P]
+            L.pa_bm_block_tables.argtypes = [P, P, i32, P, i32, P]
+            L.pa_bm_get_stats.argtypes = [P, P]
+            for f in ("pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots",
+                      "pa_bm_append_slots", "pa_bm_block_tables", "pa_bm_get_stats"):
+                getattr(L, f).restype = ctypes.c_int
+            L.pa_bm_refcount.argtypes = [P, i32]
+            L.pa_bm_refcount.restype = i32
             L.pa_status_string.argtypes = [ctypes.c_int]
             L.pa_status_string.restype = ctypes.c_char_p
             L.pa_last_cuda_error.argtypes = []
@@ -223,3 +245,81 @@ def swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping: torch.Tensor, *,
                               dst_k[0].shape[0], _dtype_code(src_k[0]), _ptr(dev_error),
                               _stream(stream, dev))
     _check(st, "pa_swap_blocks")
+
+
+class _BmStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("num_blocks", "free_blocks", "used_blocks",
+                                              "shared_blocks", "sequences", "tokens",
+                                              "logical_blocks")]
+
+
+class BlockManager:
+    """Host block manager of libpa (pa_bm_*): reference-counted 16-token
+    blocks, on-demand allocation, copy-on-write on the first divergent write.
+    Produces the host arrays the kernels consume (slot mapping, copy pairs,
+    block tables, context lengths)."""
+
+    def __init__(self, num_blocks: int, block_size: int = PA_BLOCK_SIZE):
+        self._L = lib()
+        self._h = self._L.pa_bm_create(int(num_blocks), int(block_size))
+        if not self._h:
+            raise PaError(PA_ERR_INVALID_ARG, "pa_bm_create")
+        self.num_blocks = int(num_blocks)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._L.pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    @property
+    def num_free(self) -> int:
+        return int(self._L.pa_bm_num_free_blocks(self._h))
+
+    def add_sequence(self, seq_id: int, num_tokens: int) -> None:
+        _check(self._L.pa_bm_add_sequence(self._h, int(seq_id), int(num_tokens)), "pa_bm_add_sequence")
+
+    def fork(self, parent_id: int, child_id: int) -> None:
+        _check(self._L.pa_bm_fork(self._h, int(parent_id), int(child_id)), "pa_bm_fork")
+
+    def free(self, seq_id: int) -> None:
+        _check(self._L.pa_bm_free_sequence(self._h, int(seq_id)), "pa_bm_free_sequence")
+
+    def slots(self, seq_id: int, start: int, count: int):
+        import numpy as np
+        out = np.empty(max(int(count), 0), dtype=np.int64)
+        _check(self._L.pa_bm_slots(self._h, int(seq_id), int(start), int(count),
+                                   out.ctypes.data if count > 0 else None), "pa_bm_slots")
+        return out
+
+    def append_slots(self, seq_ids):
+        """Reserve the next token's slot of each sequence. Returns
+        (slot_mapping int64 [n], cow_pairs int64 [k, 2])."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = np.empty(n, dtype=np.int64)
+        cow = np.empty((max(n, 1), 2), dtype=np.int64)
+        nc = ctypes.c_int32(0)
+        _check(self._L.pa_bm_append_slots(self._h, ids.ctypes.data, n, slots.ctypes.data,
+                                          cow.ctypes.data, ctypes.byref(nc)), "pa_bm_append_slots")
+        return slots, cow[:nc.value].copy()
+
+    def block_tables(self, seq_ids, stride: int):
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        bt = np.empty((ids.size, int(stride)), dtype=np.int32)
+        lens = np.empty(ids.size, dtype=np.int32)
+        _check(self._L.pa_bm_block_tables(self._h, ids.ctypes.data, ids.size, bt.ctypes.data,
+                                          int(stride), lens.ctypes.data), "pa_bm_block_tables")
+        return bt, lens
+
+    def stats(self) -> dict:
+        st = _BmStats()
+        _check(self._L.pa_bm_get_stats(self._h, ctypes.byref(st)), "pa_bm_get_stats")
+        return {n: int(getattr(st, n)) for n, _ in _BmStats._fields_}
+
+    def refcount(self, block: int) -> int:
+        return int(self._L.pa_bm_refcount(self._h, int(block)))
