@@ -44,6 +44,10 @@ WORKLOAD_TEXT = {
                      "1 partial CoW-forked per seq), suffix U[16,512], H_q=32, H_kv=8, D=128, bf16",
     "long": "long-context 70B-shaped GQA decode, 1 layer: batch 8, H_q=64, H_kv=8, D=128, bf16, "
             "ctx U[32768,131072], split-K 512-token partitions + LSE reduce",
+    "spec_verify": "speculative verify on the Llama-3-8B GQA batch: 256 seqs, 4 draft tokens each "
+                   "(causal in the chunk), H_q=32, H_kv=8, D=128, bf16, ctx lognormal(1024, 1)",
+    "chunked_prefill": "chunked prefill, Llama-3-8B shape: 16 prompts of U[1024,8192] tokens, "
+                       "next 256-token chunk each, H_q=32, H_kv=8, D=128, bf16",
 }
 
 
@@ -106,6 +110,9 @@ def recorded_traffic(workload: str, batch):
     return None
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -113,6 +120,28 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s, burst); fp16 has the same nominal rate."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def attention_flops(w) -> float:
+    """Multiply-adds of q.K and P.V: 4 * D flops per (query row, head, key seen)."""
+    L = w.context_lens.astype(np.int64)
+    if w.q_start is None:
+        keys = L.sum()
+    else:
+        tq = np.diff(w.q_start).astype(np.int64)
+        # query t of a chunk of tq at the end of L sees L - tq + t + 1 keys
+        keys = int((tq * (L - tq) + tq * (tq + 1) // 2).sum())
+    return 4.0 * w.head_dim * w.num_q_heads * float(keys)
 
 
 # --------------------------------------------------------------------------- clocks
@@ -239,6 +268,8 @@ class PackedInputs:
         parts = [("q", w.q.view(np.int16)), ("new_k", w.new_k.view(np.int16)),
                  ("new_v", w.new_v.view(np.int16)), ("slots", w.slot_mapping),
                  ("pairs", w.copy_pairs), ("bt", w.block_tables), ("cl", w.context_lens)]
+        if w.q_start is not None:
+            parts.append(("q_start", w.q_start))
         self.layout, off = {}, 0
         for name, a in parts:
             a = np.ascontiguousarray(a)
@@ -285,10 +316,12 @@ def run_gpu(args, rank, world, device):
     inp = packed.views(resident)
     out = torch.empty(w.q.shape, dtype=dt, device=device)
     P = w.partition_tokens
-    ws = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, P, device)
+    n_q = int(w.q.shape[0])
+    ws = pa.alloc_workspace(n_q, w.num_q_heads, w.head_dim, w.max_context_len, P, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
     max_ctx = w.max_context_len
+    max_q = int(np.diff(w.q_start).max()) if w.q_start is not None else 1
     max_parts = 1 if (P == 0 or max_ctx <= P) else -(-max_ctx // P)
     launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + \
         1 + (1 if max_parts > 1 else 0)
@@ -302,9 +335,14 @@ def run_gpu(args, rank, world, device):
                     stream=stream)
         if e_dec is not None:
             e_dec[0].record(stream)
-        pa.decode(o, x["q"], k_cache, v_cache, x["bt"], x["cl"], scale=w.scale,
-                  max_context_len=max_ctx, partition_tokens=P, workspace=ws, dev_error=err,
-                  stream=stream)
+        if "q_start" in x:
+            pa.prefill_chunk(o, x["q"], x["q_start"], k_cache, v_cache, x["bt"], x["cl"],
+                             scale=w.scale, max_query_len=max_q, max_context_len=max_ctx,
+                             partition_tokens=P, workspace=ws, dev_error=err, stream=stream)
+        else:
+            pa.decode(o, x["q"], k_cache, v_cache, x["bt"], x["cl"], scale=w.scale,
+                      max_context_len=max_ctx, partition_tokens=P, workspace=ws, dev_error=err,
+                      stream=stream)
         if e_dec is not None:
             e_dec[1].record(stream)
 
@@ -557,9 +595,12 @@ def main():
         e2e["ms"] = agg["e2e_ms"]
 
     peak, peak_src = measured_peaks()
+    tpeak, tpeak_src = measured_tensor_peak()
     K = args.steps
     value = kv_total * K / (elapsed_ms / 1e3) / 1e9
     dec_achieved = sb["decode"] / (dec_ms / 1e3) / 1e9
+    flops = attention_flops(w)
+    tensor_bound = flops / (tpeak * 1e12) > sb["decode"] / (peak * 1e9)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -588,13 +629,19 @@ def main():
         "seq_steps_per_s": round(seqs_total * K / (elapsed_ms / 1e3), 1),
         "hbm_frac_of_peak": round(value / peak, 4),
         "roofline": {
-            "kernel": "pa_decode (decode_partition_kernel + lse_reduce_kernel)",
-            "bound": "hbm",
-            "achieved": round(dec_achieved, 1),
-            "peak": peak,
-            "peak_source": peak_src,
-            "unit": "GB/s",
-            "frac": round(dec_achieved / peak, 4),
+            "kernel": ("pa_prefill_chunk" if w.q_start is not None else "pa_decode") +
+                      " (decode_partition_kernel + lse_reduce_kernel)",
+            "bound": "tensor" if tensor_bound else "hbm",
+            "achieved": round(flops / (dec_ms / 1e3) / 1e12, 2) if tensor_bound
+            else round(dec_achieved, 1),
+            "peak": tpeak if tensor_bound else peak,
+            "peak_source": tpeak_src if tensor_bound else peak_src,
+            "unit": "TFLOP/s" if tensor_bound else "GB/s",
+            "frac": round(flops / (dec_ms / 1e3) / 1e12 / tpeak, 4) if tensor_bound
+            else round(dec_achieved / peak, 4),
+            "kv_gbs": round(dec_achieved, 1),
+            "tflops": round(flops / (dec_ms / 1e3) / 1e12, 2),
+            "flops_per_launch": flops,
             "algorithmic_bytes_per_launch": sb["decode"],
             "traffic": recorded_traffic(args.workload, args.batch),
             "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "

@@ -134,6 +134,39 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     int32_t* dev_error, pa_dtype dtype, void* stream);
 
 /*
+ * Attention of several query tokens per sequence over the paged cache, causal
+ * within the chunk: the query tokens of sequence s are q rows q_start[s] ..
+ * q_start[s+1]-1 and are the LAST Tq = q_start[s+1] - q_start[s] tokens of its
+ * context (their K/V already written with pa_write_kv); query token t (0-based
+ * in the chunk) attends to context positions 0 .. context_lens[s] - Tq + t.
+ * This is the attention of chunked prefill ("PagedAttention in Action ...",
+ * "Chunked Prefill: Don't Let Long Prompts Consume the Entire Budget") and of
+ * verifying speculative draft tokens ("The Memory Wall ...", "The Next
+ * Frontier: Speculative Decoding and Beyond"). With one token per sequence it
+ * equals pa_decode.
+ *   out, q          device, [num_q_tokens][num_q_heads][head_dim]
+ *   q_start         device int32 [num_seqs + 1], non-decreasing, q_start[0] = 0
+ *   max_query_len   host upper bound of Tq (sizes the launch); Tq must also be
+ *                   <= context_lens[s]
+ *   workspace       >= pa_decode_workspace_size(num_q_tokens, num_q_heads,
+ *                   head_dim, max_context_len, partition_tokens) bytes
+ *   other arguments as for pa_decode. A sequence whose query range falls
+ *   outside [0, num_q_tokens) is skipped, one whose Tq exceeds max_query_len
+ *   or its context length is clamped; both are counted in dev_error. With a
+ *   malformed q_start the output rows of the sequences involved are undefined
+ *   (never written out of bounds).
+ */
+pa_status pa_prefill_chunk(void* out, const void* q, const int32_t* q_start,
+                           int32_t num_q_tokens, int32_t max_query_len, const void* k_cache,
+                           const void* v_cache, const int32_t* block_tables,
+                           int32_t block_table_stride, const int32_t* context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t group_size,
+                           int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                           int32_t max_context_len, float scale, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                           pa_dtype dtype, void* stream);
+
+/*
  * Copy-on-write block copies: for each pair p and each layer l,
  * k_caches[l][dst] = k_caches[l][src] and v_caches[l][dst] = v_caches[l][src]
  * (whole blocks: num_kv_heads * 16 * head_dim elements), src = mapping[2p],

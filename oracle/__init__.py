@@ -16,6 +16,10 @@ What each function follows, by page and section:
   is copied when one sequence diverges, the shared original stays unchanged.
 * ``swap_blocks`` -- "PagedAttention", "Managing Virtual Memory (Block
   Manager)": blocks move between GPU memory and CPU RAM and back.
+* ``prefill_chunk`` -- "PagedAttention in Action ...", "Chunked Prefill", and
+  "The Memory Wall ...", "The Next Frontier: Speculative Decoding and Beyond":
+  the last Tq tokens of a context are queries at once, each seeing the context
+  up to its own position.
 * ``decode`` -- same first page, "PagedAttention: Decoupling Logical Context
   from Contiguous GPU Memory" (Figure 2), and "The Memory Wall ...", "How it
   Works Under the Hood" and "Show Me The Code": the kernel walks the block
@@ -170,3 +174,25 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype,
     if rc != 0:
         raise ValueError("oracle.decode: a block-table entry is outside [0, num_blocks)")
     return out
+
+
+def prefill_chunk(q, q_start, k_cache, v_cache, block_tables, context_lens, scale: float, dtype,
+                  rows=None, n_threads: int = 0) -> np.ndarray:
+    """Attention of each sequence's last Tq context tokens, causal in the chunk.
+
+    ``q``: uint16 bits ``[T, H_q, D]`` where sequence s owns rows
+    ``q_start[s] .. q_start[s+1]-1``. Query token t of sequence s (t counted
+    from the chunk start) attends to context positions
+    ``0 .. context_lens[s] - Tq_s + t`` -- i.e. it is the decode of one query
+    over the first ``context_lens[s] - Tq_s + t + 1`` tokens of the same
+    block table. Returns ``[T, H_q, D]`` float64 (or the requested flat
+    ``token * H_q + head`` rows)."""
+    q_start = np.asarray(q_start, dtype=np.int64)
+    context_lens = np.asarray(context_lens, dtype=np.int64)
+    block_tables = np.asarray(block_tables, dtype=np.int32)
+    tq = np.diff(q_start)
+    tok_seq = np.repeat(np.arange(len(tq)), tq)
+    tok_t = np.arange(int(q_start[-1])) - q_start[tok_seq]
+    tok_len = (context_lens[tok_seq] - tq[tok_seq] + tok_t + 1).astype(np.int32)
+    return decode(q, k_cache, v_cache, block_tables[tok_seq], tok_len, scale, dtype, rows=rows,
+                  n_threads=n_threads)

@@ -146,7 +146,15 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
   return round256(rows * head_dim * sizeof(float)) + round256(rows * sizeof(float));
 }
 
-pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+}  // extern "C"
+
+namespace {
+
+// The common body of pa_decode (q_start == NULL: one query token per
+// sequence) and pa_prefill_chunk (q_start[s] .. q_start[s + 1] are the query
+// tokens of sequence s, the last ones of its context).
+pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t num_q_tokens,
+                    int32_t max_query_len, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int32_t block_table_stride,
                     const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
                     int32_t group_size, int32_t head_dim, int32_t block_size,
@@ -154,28 +162,32 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                     int32_t* dev_error, pa_dtype dtype, void* stream) {
   if (num_seqs < 0 || num_q_heads < 1 || group_size < 1 || num_blocks < 1 ||
-      max_context_len < 0 || partition_tokens < 0 || !valid_dtype(dtype) || !isfinite(scale))
+      max_context_len < 0 || partition_tokens < 0 || !valid_dtype(dtype) || !isfinite(scale) ||
+      num_q_tokens < 0 || max_query_len < 0)
     return PA_ERR_INVALID_ARG;
   if (block_size != PA_BLOCK_SIZE || (head_dim != 64 && head_dim != 128) || group_size > 16 ||
       num_q_heads % group_size != 0 || partition_tokens % PA_BLOCK_SIZE != 0)
     return PA_ERR_UNSUPPORTED;
   const int32_t num_kv_heads = num_q_heads / group_size;
   if (num_seqs > 65535 || num_kv_heads > 65535 || num_blocks > (int64_t(1) << 32) ||
-      (int64_t)num_seqs * num_q_heads > 0x7fffffff)
+      (int64_t)num_q_tokens * num_q_heads > 0x7fffffff)
     return PA_ERR_UNSUPPORTED;
-  if (num_seqs == 0) return PA_OK;
+  if (num_seqs == 0 || num_q_tokens == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return PA_ERR_INVALID_ARG;
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(block_tables, 4) || !aligned(context_lens, 4) || (dev_error && !aligned(dev_error, 4)))
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || (dev_error && !aligned(dev_error, 4)) ||
+      (q_start && !aligned(q_start, 4)))
     return PA_ERR_INVALID_ARG;
   const int64_t max_blocks = ((int64_t)max_context_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE;
   if (block_table_stride < max_blocks || block_table_stride < 1) return PA_ERR_INVALID_ARG;
 
   const int64_t parts = max_partitions(max_context_len, partition_tokens);
-  if (parts > 0x7fffffff) return PA_ERR_UNSUPPORTED;
-  const size_t need =
-      pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens);
+  const int64_t qtiles = q_start ? ((int64_t)max_query_len * group_size + 15) / 16 : 1;
+  if (qtiles < 1) return PA_OK;  // no query token can exist
+  if (parts * qtiles > 0x7fffffff) return PA_ERR_UNSUPPORTED;
+  const size_t need = pa_decode_workspace_size(num_q_tokens, num_q_heads, head_dim,
+                                               max_context_len, partition_tokens);
   if (need > 0) {
     if (!workspace || !aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
     if (workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
@@ -186,13 +198,17 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   if (st != PA_OK) return st;
   st = encode_pool_map(&a.tm_v, v_cache, num_blocks, num_kv_heads, head_dim, dtype);
   if (st != PA_OK) return st;
-  const size_t rows = (size_t)num_seqs * num_q_heads * parts;
+  const size_t rows = (size_t)num_q_tokens * num_q_heads * parts;
   a.out = out;
   a.part_o = need ? static_cast<float*>(workspace) : nullptr;
   a.part_lse = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                round256(rows * head_dim * sizeof(float)))
                     : nullptr;
   a.q = q;
+  a.q_start = q_start;
+  a.num_q_tokens = num_q_tokens;
+  a.max_query_len = q_start ? max_query_len : 1;
+  a.max_qtiles = (int32_t)qtiles;
   a.block_tables = block_tables;
   a.bt_stride = block_table_stride;
   a.context_lens = context_lens;
@@ -212,6 +228,39 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   a.bf16 = dtype == PA_DTYPE_BF16;
   cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t block_table_stride,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t group_size, int32_t head_dim, int32_t block_size,
+                    int64_t num_blocks, int32_t max_context_len, float scale,
+                    int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_error, pa_dtype dtype, void* stream) {
+  return attention(out, q, nullptr, num_seqs, 1, k_cache, v_cache, block_tables,
+                   block_table_stride, context_lens, num_seqs, num_q_heads, group_size, head_dim,
+                   block_size, num_blocks, max_context_len, scale, partition_tokens, workspace,
+                   workspace_bytes, dev_error, dtype, stream);
+}
+
+pa_status pa_prefill_chunk(void* out, const void* q, const int32_t* q_start,
+                           int32_t num_q_tokens, int32_t max_query_len, const void* k_cache,
+                           const void* v_cache, const int32_t* block_tables,
+                           int32_t block_table_stride, const int32_t* context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t group_size,
+                           int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                           int32_t max_context_len, float scale, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                           pa_dtype dtype, void* stream) {
+  if (!q_start) return PA_ERR_INVALID_ARG;
+  return attention(out, q, q_start, num_q_tokens, max_query_len, k_cache, v_cache, block_tables,
+                   block_table_stride, context_lens, num_seqs, num_q_heads, group_size, head_dim,
+                   block_size, num_blocks, max_context_len, scale, partition_tokens, workspace,
+                   workspace_bytes, dev_error, dtype, stream);
 }
 
 pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_layers,

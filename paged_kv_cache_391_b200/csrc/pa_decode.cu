@@ -74,16 +74,22 @@ __device__ __forceinline__ uint32_t tile_off(int t, int d) {
   return (uint32_t)((d >> 6) * 2048 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4) + (d & 7) * 2);
 }
 
-template <typename T, int D, bool kTwoRows>
+// kMulti = false: one query token per sequence (decode); the tile's rows are
+// the query heads of one KV head. kMulti = true: each sequence's last Tq
+// context tokens are queries (a prompt chunk, or speculative draft tokens);
+// the tile's rows are (query token, head) pairs, 16 per tile, and query token
+// t sees the context up to its own position L - Tq + t (causal in the chunk).
+template <typename T, int D, bool kTwoRows, bool kMulti>
 __global__ void __launch_bounds__(kThreads)
     decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, T* __restrict__ out,
                             float* __restrict__ part_o, float* __restrict__ part_lse,
-                            const T* __restrict__ q, const int32_t* __restrict__ block_tables,
-                            int bt_stride, const int32_t* __restrict__ context_lens,
-                            int num_q_heads, int group, int64_t num_blocks, int max_context_len,
-                            float scale_log2, int part_blocks, int max_parts,
-                            int32_t* __restrict__ dev_error) {
+                            const T* __restrict__ q, const int32_t* __restrict__ q_start,
+                            int num_q_tokens, int max_query_len,
+                            const int32_t* __restrict__ block_tables, int bt_stride,
+                            const int32_t* __restrict__ context_lens, int num_q_heads, int group,
+                            int64_t num_blocks, int max_context_len, float scale_log2,
+                            int part_blocks, int max_parts, int32_t* __restrict__ dev_error) {
   using SM = DecodeSmem<D>;
   using E = Elem<T>;
   extern __shared__ uint8_t smem_raw[];
@@ -91,21 +97,49 @@ __global__ void __launch_bounds__(kThreads)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOffset);
 
-  const int part = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int kvh = blockIdx.y, seq = blockIdx.z;
+  const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x;
+  const int qtile = kMulti ? (int)(blockIdx.x / (unsigned)max_parts) : 0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
+  const bool counter = part == 0 && kvh == 0 && qtile == 0 && tid == 0 && dev_error;
 
   int L = context_lens[seq];
   if (L < 0 || L > max_context_len) {
-    if (part == 0 && kvh == 0 && tid == 0 && dev_error) atomicAdd(dev_error, 1);
+    if (counter) atomicAdd(dev_error, 1);
     L = L < 0 ? 0 : max_context_len;
   }
+  // Query rows of this sequence: q0 = first query token, Tq tokens.
+  int q0 = seq, Tq = 1;
+  if (kMulti) {
+    q0 = q_start[seq];
+    Tq = q_start[seq + 1] - q0;
+    if (q0 < 0 || Tq < 0 || q0 + Tq > num_q_tokens) {
+      if (counter) atomicAdd(dev_error, 1);  // query range outside the q buffer: skip
+      return;
+    }
+    const int cap = min(L, max_query_len);
+    if (Tq > cap) {
+      if (counter) atomicAdd(dev_error, 1);
+      Tq = cap;
+    }
+  }
+  const int rows_total = Tq * group;
+  const int row0 = qtile * 16;
+  if (row0 >= rows_total) return;
+  const int nrows = min(16, rows_total - row0);  // rows of this tile (decode: = group)
+
   const int nblk_seq = (L + kBlockTokens - 1) / kBlockTokens;
   const int n_parts = nblk_seq > 0 ? (nblk_seq + part_blocks - 1) / part_blocks : 1;
   if (part >= n_parts) return;
   const int blk_begin = part * part_blocks;
   const int nblk = min(nblk_seq - blk_begin, part_blocks);  // 0 only for an empty context
   const int q_head0 = kvh * group;
+  // This lane's two tile rows (a = gid, b = gid + 8): query token and head.
+  const int ta = (row0 + gid) / group, ha = (row0 + gid) - ta * group;
+  const int tb = (row0 + gid + 8) / group, hb = (row0 + gid + 8) - tb * group;
+  const int lim_a = L - Tq + ta;  // last key position row a may attend to
+  const int lim_b = L - Tq + tb;
 
   // ---- this warp's share: blocks blk_begin + warp + kWarps * it
   const int n_mine = nblk > warp ? (nblk - warp + kWarps - 1) / kWarps : 0;
@@ -170,12 +204,12 @@ __global__ void __launch_bounds__(kThreads)
   uint32_t qa[D / 16][4];
   {
     const uint32_t* qa_row =
-        gid < group ? reinterpret_cast<const uint32_t*>(
-                          q + ((size_t)seq * num_q_heads + q_head0 + gid) * D)
+        gid < nrows ? reinterpret_cast<const uint32_t*>(
+                          q + ((size_t)(q0 + ta) * num_q_heads + q_head0 + ha) * D)
                     : nullptr;
     const uint32_t* qb_row =
-        (kTwoRows && gid + 8 < group)
-            ? reinterpret_cast<const uint32_t*>(q + ((size_t)seq * num_q_heads + q_head0 + gid + 8) * D)
+        (kTwoRows && gid + 8 < nrows)
+            ? reinterpret_cast<const uint32_t*>(q + ((size_t)(q0 + tb) * num_q_heads + q_head0 + hb) * D)
             : nullptr;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -237,8 +271,12 @@ __global__ void __launch_bounds__(kThreads)
 
       // Online softmax (base 2). Lane holds, for head row a = gid (and
       // b = gid + 8), tokens 2tig, 2tig+1 (s0) and 8+2tig, 9+2tig (s1).
+      // Keys of this block row a (b) may see: the context, and in a chunk
+      // only up to the row's own position.
       const int t0 = 2 * tig;
-      const bool v0 = t0 < valid, v1 = t0 + 1 < valid, v2 = t0 + 8 < valid, v3 = t0 + 9 < valid;
+      const int na = kMulti ? min(valid, lim_a - j * kBlockTokens + 1) : valid;
+      const int nb = kMulti ? min(valid, lim_b - j * kBlockTokens + 1) : valid;
+      bool v0 = t0 < na, v1 = t0 + 1 < na, v2 = t0 + 8 < na, v3 = t0 + 9 < na;
       uint32_t pa[4];
       {
         const float x0 = v0 ? s0[0] * scale_log2 : -INFINITY;
@@ -263,6 +301,7 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
       if (kTwoRows) {
+        v0 = t0 < nb, v1 = t0 + 1 < nb, v2 = t0 + 8 < nb, v3 = t0 + 9 < nb;
         const float x0 = v0 ? s0[2] * scale_log2 : -INFINITY;
         const float x1 = v1 ? s0[3] * scale_log2 : -INFINITY;
         const float x2 = v2 ? s1[2] * scale_log2 : -INFINITY;
@@ -324,7 +363,7 @@ __global__ void __launch_bounds__(kThreads)
   float* mo = reinterpret_cast<float*>(smem);
   float* mm = mo + kWarps * 16 * SM::kMergeStride;
   float* ml = mm + kWarps * 16;
-  if (gid < group) {
+  if (gid < nrows) {
     float* row = mo + (warp * 16 + gid) * SM::kMergeStride;
 #pragma unroll
     for (int n = 0; n < D / 8; ++n)
@@ -334,7 +373,7 @@ __global__ void __launch_bounds__(kThreads)
       ml[warp * 16 + gid] = l_a;
     }
   }
-  if (kTwoRows && gid + 8 < group) {
+  if (kTwoRows && gid + 8 < nrows) {
     float* row = mo + (warp * 16 + gid + 8) * SM::kMergeStride;
 #pragma unroll
     for (int n = 0; n < D / 8; ++n)
@@ -347,8 +386,8 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
 
   const bool direct = n_parts == 1;
-  for (int idx = tid; idx < group * (D / 4); idx += kThreads) {
-    const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
+  for (int idx = tid; idx < nrows * (D / 4); idx += kThreads) {
+    const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;  // h: tile row
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * 16 + h]);
@@ -373,7 +412,8 @@ __global__ void __launch_bounds__(kThreads)
       res.z = acc.z / lsum;
       res.w = acc.w / lsum;
     }
-    const size_t orow = (size_t)seq * num_q_heads + q_head0 + h;
+    const int t = (row0 + h) / group;
+    const size_t orow = (size_t)(q0 + t) * num_q_heads + q_head0 + (row0 + h - t * group);
     if (direct) {
       uint2 pk;
       pk.x = E::pack(res.x, res.y);
@@ -392,14 +432,29 @@ __global__ void __launch_bounds__(kThreads)
 // first (max and sum in a fixed order), then independent weighted loads.
 // Deterministic: the summation order depends only on the partition count.
 constexpr int kReduceWarps = 8;
+
+// Sequence of an output row: rows are (query token, head); with one token per
+// sequence the token is the sequence, otherwise q_start (the first token of
+// each sequence, num_seqs + 1 entries) is searched.
+__device__ __forceinline__ int seq_of_row(int row, int num_q_heads, const int32_t* q_start,
+                                          int num_seqs) {
+  const int token = row / num_q_heads;
+  if (!q_start) return token;
+  int lo = 0, hi = num_seqs - 1;  // last seq with q_start[seq] <= token
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (q_start[mid] <= token) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
 constexpr int kWarpRowMaxParts = 16;  // up to this many, one warp (half-warp) per row
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
     lse_reduce_kernel(T* __restrict__ out, const float* __restrict__ part_o,
                       const float* __restrict__ part_lse, const int32_t* __restrict__ context_lens,
-                      int num_rows, int num_q_heads, int max_context_len, int part_tokens,
-                      int max_parts) {
+                      const int32_t* __restrict__ q_start, int num_seqs, int num_rows,
+                      int num_q_heads, int max_context_len, int part_tokens, int max_parts) {
   constexpr int kLanes = D / 4;             // float4 columns of a row = lanes per row
   constexpr int kRowsPerWarp = 32 / kLanes;
   using E = Elem<T>;
@@ -409,7 +464,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   const unsigned grp = kRowsPerWarp == 1 ? kFull : (0xffffu << (lane & ~(kLanes - 1)));
   int n = 0;
   if (row < num_rows) {
-    int L = context_lens[row / num_q_heads];
+    int L = context_lens[seq_of_row(row, num_q_heads, q_start, num_seqs)];
     L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
     n = (L + part_tokens - 1) / part_tokens;
   }
@@ -460,7 +515,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
     lse_reduce_split_kernel(T* __restrict__ out, const float* __restrict__ part_o,
                             const float* __restrict__ part_lse,
-                            const int32_t* __restrict__ context_lens, int num_q_heads,
+                            const int32_t* __restrict__ context_lens,
+                            const int32_t* __restrict__ q_start, int num_seqs, int num_q_heads,
                             int max_context_len, int part_tokens, int max_parts) {
   constexpr int kThreadsR = kReduceWarps * 32;
   constexpr int kLanes = D / 4;
@@ -470,7 +526,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   __shared__ float s_red[kThreadsR];
   __shared__ float4 s_acc[kStreams][kLanes];
   const int row = blockIdx.x;
-  int L = context_lens[row / num_q_heads];
+  int L = context_lens[seq_of_row(row, num_q_heads, q_start, num_seqs)];
   L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
   const int n = (L + part_tokens - 1) / part_tokens;
   if (n <= 1) return;
@@ -546,20 +602,21 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   }
 }
 
-template <typename T, int D, bool kTwoRows>
+template <typename T, int D, bool kTwoRows, bool kMulti>
 static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
   using SM = DecodeSmem<D>;
-  auto kern = decode_partition_kernel<T, D, kTwoRows>;
+  auto kern = decode_partition_kernel<T, D, kTwoRows, kMulti>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.max_parts, a.num_kv_heads, a.num_seqs);
+  dim3 grid((unsigned)((int64_t)a.max_parts * a.max_qtiles), a.num_kv_heads, a.num_seqs);
   kern<<<grid, kThreads, SM::kAlloc, stream>>>(
       a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, static_cast<const T*>(a.q),
-      a.block_tables, a.bt_stride, a.context_lens, a.num_q_heads, a.group, a.num_blocks,
-      a.max_context_len, a.scale_log2, a.part_blocks, a.max_parts, a.dev_error);
+      a.q_start, a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride, a.context_lens,
+      a.num_q_heads, a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
+      a.max_parts, a.dev_error);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.max_parts <= 1) return e;
-  const int rows = a.num_seqs * a.num_q_heads;
+  const int rows = a.num_q_tokens * a.num_q_heads;
   if (a.max_parts > kWarpRowMaxParts) {
     const size_t wbytes = (size_t)a.max_parts * sizeof(float);
     if (wbytes > 48 * 1024) {
@@ -568,24 +625,31 @@ static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
       if (e != cudaSuccess) return e;
     }
     lse_reduce_split_kernel<T, D><<<rows, kReduceWarps * 32, wbytes, stream>>>(
-        static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.num_q_heads,
-        a.max_context_len, a.part_tokens, a.max_parts);
+        static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start, a.num_seqs,
+        a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts);
   } else {
     const int rows_per_cta = kReduceWarps * (32 / (D / 4));
     lse_reduce_kernel<T, D><<<(rows + rows_per_cta - 1) / rows_per_cta, kReduceWarps * 32, 0,
                               stream>>>(static_cast<T*>(a.out), a.part_o, a.part_lse,
-                                        a.context_lens, rows, a.num_q_heads, a.max_context_len,
-                                        a.part_tokens, a.max_parts);
+                                        a.context_lens, a.q_start, a.num_seqs, rows,
+                                        a.num_q_heads, a.max_context_len, a.part_tokens,
+                                        a.max_parts);
   }
   return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_dtype(const DecodeLaunch& a, cudaStream_t stream) {
+  if (a.q_start) {  // query chunks: tiles mix tokens and heads, both row halves in use
+    return a.head_dim == 128 ? launch_typed<T, 128, true, true>(a, stream)
+                             : launch_typed<T, 64, true, true>(a, stream);
+  }
   const bool two = a.group > 8;
   if (a.head_dim == 128)
-    return two ? launch_typed<T, 128, true>(a, stream) : launch_typed<T, 128, false>(a, stream);
-  return two ? launch_typed<T, 64, true>(a, stream) : launch_typed<T, 64, false>(a, stream);
+    return two ? launch_typed<T, 128, true, false>(a, stream)
+               : launch_typed<T, 128, false, false>(a, stream);
+  return two ? launch_typed<T, 64, true, false>(a, stream)
+             : launch_typed<T, 64, false, false>(a, stream);
 }
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {

@@ -18,6 +18,10 @@ struct DecodeLaunch {
   float* part_o;     // [S][H_q][max_parts][D]
   float* part_lse;   // [S][H_q][max_parts]
   const void* q;
+  const int32_t* q_start;  // NULL: one query token per sequence (decode)
+  int32_t num_q_tokens;    // rows of q / out (= num_seqs for decode)
+  int32_t max_query_len;   // 1 for decode
+  int32_t max_qtiles;      // 16-row query tiles per (sequence, KV head)
   const int32_t* block_tables;
   int32_t bt_stride;
   const int32_t* context_lens;

@@ -27,7 +27,7 @@ EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_bloc
            "pa_status_string", "pa_last_cuda_error", "pa_decode_static", "pa_swap_blocks",
            "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence",
            "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots", "pa_bm_append_slots",
-           "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount")
+           "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount", "pa_prefill_chunk")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
             L.pa_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, i32,
                                     ctypes.c_float, i32, P, sz, P, ctypes.c_int, P]
             L.pa_decode.restype = ctypes.c_int
+            L.pa_prefill_chunk.argtypes = [P, P, P, i32, i32, P, P, P, i32, P, i32, i32, i32,
+                                           i32, i32, i64, i32, ctypes.c_float, i32, P, sz, P,
+                                           ctypes.c_int, P]
+            L.pa_prefill_chunk.restype = ctypes.c_int
             L.pa_decode_static.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                            i32, ctypes.c_float, i32, P, ctypes.c_int, P]
             L.pa_decode_static.restype = ctypes.c_int
@@ -181,6 +185,36 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
                          int(partition_tokens), _ptr(workspace), ws_bytes, _ptr(dev_error),
                          _dtype_code(q), _stream(stream, q.device))
     _check(st, "pa_decode")
+    return out
+
+
+def prefill_chunk(out: torch.Tensor, q: torch.Tensor, q_start: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, *,
+                  scale: float, max_query_len: int, max_context_len: int,
+                  partition_tokens: int = 512, workspace: torch.Tensor | None = None,
+                  dev_error: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Attention of each sequence's last Tq context tokens (rows
+    ``q_start[s]:q_start[s+1]`` of ``q [T, H_q, D]``), causal within the chunk:
+    chunked prefill or speculative-draft verification over the paged cache."""
+    T, Hq, D = q.shape
+    NB, Hkv = k_cache.shape[:2]
+    S = context_lens.numel()
+    assert out.shape == q.shape and out.dtype == q.dtype == k_cache.dtype == v_cache.dtype
+    assert k_cache.shape == v_cache.shape == (NB, Hkv, PA_BLOCK_SIZE, D)
+    assert q_start.dtype == torch.int32 and q_start.numel() == S + 1
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    if Hq % Hkv:
+        raise ValueError("num_q_heads must be a multiple of num_kv_heads")
+    if workspace is None:
+        workspace = alloc_workspace(T, Hq, D, max_context_len, partition_tokens, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().pa_prefill_chunk(_ptr(out), _ptr(q), _ptr(q_start), T, int(max_query_len),
+                                _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                block_tables.shape[1], _ptr(context_lens), S, Hq, Hq // Hkv, D,
+                                PA_BLOCK_SIZE, NB, int(max_context_len), float(scale),
+                                int(partition_tokens), _ptr(workspace), ws_bytes,
+                                _ptr(dev_error), _dtype_code(q), _stream(stream, q.device))
+    _check(st, "pa_prefill_chunk")
     return out
 
 

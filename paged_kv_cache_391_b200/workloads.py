@@ -59,6 +59,7 @@ class DecodeWorkload:
     seed: int = 0
     notes: dict = field(default_factory=dict)
     block_size: int = BLOCK_SIZE
+    q_start: np.ndarray | None = None  # int32 [S+1] for query chunks; None = one token each
 
     @property
     def num_seqs(self) -> int:
@@ -103,8 +104,9 @@ class DecodeWorkload:
         T = int(self.slot_mapping.shape[0])
         n_pairs = int(self.copy_pairs.shape[0])
         blk = Hkv * self.block_size * D * self.elem_bytes
+        Tq = int(self.q.shape[0])  # query rows: S for decode, sum of chunk lengths otherwise
         return {
-            "decode": self.kv_bytes() + 2 * S * Hq * D * self.elem_bytes
+            "decode": self.kv_bytes() + 2 * Tq * Hq * D * self.elem_bytes
             + S * 4 + int((np.ceil(self.context_lens / self.block_size)).sum()) * 4,
             "write_kv": 2 * 2 * T * Hkv * D * self.elem_bytes + T * 8,
             "copy_blocks": 2 * 2 * n_pairs * blk + n_pairs * 16,
@@ -246,6 +248,53 @@ def decode_workload(name: str, context_lens, *, num_q_heads: int, num_kv_heads: 
                   {"pool_factor": pool_factor, "blocks_used": int(sum(need))})
 
 
+def chunk_workload(name: str, context_lens, query_lens, *, num_q_heads: int, num_kv_heads: int,
+                   head_dim: int, dtype: str, seed: int, pool_factor: float = 1.5,
+                   partition_tokens: int = 512,
+                   rng: np.random.Generator | None = None) -> DecodeWorkload:
+    """Each sequence's last ``query_lens[s]`` context tokens are written this
+    step and are the queries (a prompt chunk, or draft tokens to verify);
+    ``context_lens`` counts them. q has sum(query_lens) rows, sequence s owning
+    rows ``q_start[s]:q_start[s+1]``."""
+    rng = rng if rng is not None else np.random.default_rng(seed)
+    lens = np.asarray(context_lens, dtype=np.int64)
+    tq = np.asarray(query_lens, dtype=np.int64)
+    assert (tq >= 0).all() and (tq <= lens).all()
+    need = [blocks_needed(int(L)) for L in lens]
+    nb = max(1, int(np.ceil(pool_factor * sum(need))))
+    alloc = ToyBlockAllocator(nb, rng)
+    tables = [alloc.allocate(n) for n in need]
+    writes = [(s, int(p)) for s in range(len(lens)) for p in range(int(lens[s] - tq[s]), int(lens[s]))]
+    w = _build(name, dtype, num_q_heads, num_kv_heads, head_dim, partition_tokens, seed, rng,
+               tables, _fills_for(tables, lens - tq), lens, nb, writes, [],
+               {"pool_factor": pool_factor, "query_lens": tq.tolist()})
+    w.q = _normal_bits(rng, (int(tq.sum()), num_q_heads, head_dim), dtype)
+    w.q_start = np.concatenate([[0], np.cumsum(tq)]).astype(np.int32)
+    return w
+
+
+def spec_verify(seed: int = 396, batch: int = 256, draft: int = 4) -> DecodeWorkload:
+    """Speculative-decoding verification on the Llama-3-8B-shaped GQA batch:
+    each of 256 sequences (lognormal lengths, median 1024) checks ``draft``
+    proposed tokens in one pass; with 4 query heads per KV head, 4 tokens fill
+    one 16-row tile."""
+    rng = np.random.default_rng(seed)
+    lens = np.clip(np.round(np.exp(np.log(1024.0) + rng.standard_normal(batch))),
+                   16, 8192).astype(np.int64)
+    return chunk_workload("spec_verify", lens, np.full(batch, draft), num_q_heads=32,
+                          num_kv_heads=8, head_dim=128, dtype="bf16", seed=seed, rng=rng)
+
+
+def chunked_prefill(seed: int = 397, batch: int = 16, chunk: int = 256) -> DecodeWorkload:
+    """Chunked prefill on the Llama-3-8B shape: 16 prompts of 1024..8192
+    tokens, each processing its next ``chunk`` prompt tokens against the
+    prefix already cached."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(1024, 8192, size=batch, endpoint=True)
+    return chunk_workload("chunked_prefill", lens, np.full(batch, chunk), num_q_heads=32,
+                          num_kv_heads=8, head_dim=128, dtype="bf16", seed=seed, rng=rng)
+
+
 # ---------------------------------------------------------------------------
 # The five named configurations.
 # ---------------------------------------------------------------------------
@@ -348,6 +397,8 @@ CONFIGS = {
     "gqa": gqa,
     "shared_prefix": shared_prefix,
     "long": long_context,
+    "spec_verify": spec_verify,
+    "chunked_prefill": chunked_prefill,
 }
 
 

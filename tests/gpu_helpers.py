@@ -46,8 +46,8 @@ class DeviceStep:
         self.cl = torch.from_numpy(w.context_lens).cuda()
         self.out = torch.empty(w.q.shape, dtype=dt, device="cuda")
         self.P = w.partition_tokens if partition_tokens is None else partition_tokens
-        self.ws = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len,
-                                     self.P, "cuda")
+        self.ws = pa.alloc_workspace(int(w.q.shape[0]), w.num_q_heads, w.head_dim,
+                                     w.max_context_len, self.P, "cuda")
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def cache_ops(self):
@@ -61,6 +61,17 @@ class DeviceStep:
         pa.decode(out, self.q, self.k_cache, self.v_cache, self.bt, self.cl, scale=self.w.scale,
                   max_context_len=self.w.max_context_len, partition_tokens=self.P,
                   workspace=self.ws, dev_error=self.err)
+        return out
+
+    def prefill(self, out=None):
+        """The chunk attention of a workload built by workloads.chunk_workload."""
+        out = self.out if out is None else out
+        w = self.w
+        qs = torch.from_numpy(w.q_start).cuda()
+        pa.prefill_chunk(out, self.q, qs, self.k_cache, self.v_cache, self.bt, self.cl,
+                         scale=w.scale, max_query_len=int(np.diff(w.q_start).max()),
+                         max_context_len=w.max_context_len, partition_tokens=self.P,
+                         workspace=self.ws, dev_error=self.err)
         return out
 
     def step(self):

@@ -421,3 +421,46 @@ def test_swap_blocks_between_pools_of_different_sizes():
         assert np.array_equal(dev_k[l][5], orig[l][4])
         untouched = [b for b in range(12) if b not in (11, 0, 5)]
         assert np.array_equal(dev_k[l][untouched], orig[l][untouched])
+
+
+# --------------------------------------------------------------------------
+# query chunks (chunked prefill / speculative verification)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lens,tq,Hq,Hkv,D,dtype", [
+    ([20, 5, 40], [3, 5, 1], 4, 2, 64, "f16"),
+    ([100, 37], [17, 4], 8, 2, 128, "bf16"),
+    ([64], [64], 2, 1, 64, "f16"),                 # the whole context is the chunk
+])
+def test_prefill_chunk_matches_library_attention_with_causal_mask(lens, tq, Hq, Hkv, D, dtype):
+    """Query token t of a chunk of Tq at the end of an L-token context sees
+    keys 0 .. L-Tq+t: torch's attention with that (bottom-right aligned)
+    boolean mask on the contiguous context."""
+    rng = np.random.default_rng(sum(lens) + sum(tq))
+    q, ck, cv, kp, vp, bt, cl = _random_case(rng, lens, Hq, Hkv, D, dtype)
+    q_start = np.concatenate([[0], np.cumsum(tq)]).astype(np.int32)
+    qc = _bits(rng, (int(q_start[-1]), Hq, D), dtype)
+    scale = 1 / np.sqrt(D)
+    out = oracle.prefill_chunk(qc, q_start, kp, vp, bt, cl, scale, dtype)
+    for s, (L, T) in enumerate(zip(lens, tq)):
+        K = torch.from_numpy(oracle.decode16(ck[s], dtype).transpose(1, 0, 2))[None]
+        V = torch.from_numpy(oracle.decode16(cv[s], dtype).transpose(1, 0, 2))[None]
+        Q = torch.from_numpy(oracle.decode16(qc[q_start[s]:q_start[s + 1]], dtype).transpose(1, 0, 2))[None]
+        pos_q = torch.arange(L - T, L)[:, None]
+        mask = torch.arange(L)[None, :] <= pos_q           # [T, L]
+        ref = F.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=scale,
+                                             enable_gqa=Hkv != Hq)[0].transpose(0, 1).numpy()
+        np.testing.assert_allclose(out[q_start[s]:q_start[s + 1]], ref, rtol=1e-11, atol=1e-12)
+        if T == L:   # a chunk that is the whole context is ordinary causal attention
+            ref2 = F.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=scale,
+                                                  enable_gqa=Hkv != Hq)[0].transpose(0, 1).numpy()
+            np.testing.assert_allclose(out[q_start[s]:q_start[s + 1]], ref2, rtol=1e-11, atol=1e-12)
+
+
+def test_one_token_chunks_are_decode():
+    rng = np.random.default_rng(15)
+    q, ck, cv, kp, vp, bt, cl = _random_case(rng, [9, 30, 77], 4, 2, 64, "bf16")
+    q_start = np.arange(4, dtype=np.int32)
+    a = oracle.prefill_chunk(q, q_start, kp, vp, bt, cl, 0.125, "bf16")
+    b = oracle.decode(q, kp, vp, bt, cl, 0.125, "bf16")
+    assert np.array_equal(a, b)

@@ -1,0 +1,85 @@
+"""GPU parity of pa_prefill_chunk (several query tokens per sequence, causal
+within the chunk: chunked prefill, speculative-draft verification) against
+the oracle's definition: query token t of a chunk of Tq at the end of an
+L-token context is the decode over the first L - Tq + t + 1 tokens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_391_b200 import pa
+from paged_kv_cache_391_b200 import workloads as W
+
+from gpu_helpers import (DeviceStep, assert_decode_close, host16, oracle_caches_after_step,
+                         to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(w, P=None):
+    d = DeviceStep(w, P)
+    d.cache_ops()
+    d.prefill()
+    torch.cuda.synchronize()
+    kc, vc = oracle_caches_after_step(w)
+    assert np.array_equal(host16(d.k_cache), kc) and np.array_equal(host16(d.v_cache), vc)
+    ref = oracle.prefill_chunk(w.q, w.q_start, kc, vc, w.block_tables, w.context_lens, w.scale,
+                               w.dtype)
+    assert_decode_close(to_f64(d.out), ref, w.name)
+    assert int(d.err.item()) == 0
+    return d
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (16, 2), (16, 1), (12, 1)])
+@pytest.mark.parametrize("D,dtype", [(64, "f16"), (128, "bf16")])
+def test_ragged_chunks(Hq, Hkv, D, dtype):
+    lens = [1, 16, 17, 40, 130, 600, 1100]
+    tq = [1, 16, 3, 40, 5, 33, 64]
+    w = W.chunk_workload("c", lens, tq, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                         dtype=dtype, seed=Hq * 7 + Hkv + D)
+    _check(w)
+
+
+@pytest.mark.parametrize("P", [0, 16, 128, 512])
+def test_chunk_partition_sizes(P):
+    w = W.chunk_workload("p", [700, 513, 90, 2000], [100, 9, 90, 4], num_q_heads=8,
+                         num_kv_heads=2, head_dim=128, dtype="bf16", seed=P + 3)
+    _check(w, P)
+
+
+def test_spec_verify_and_chunked_prefill_shapes():
+    _check(W.spec_verify(batch=12))
+    _check(W.chunked_prefill(batch=2, chunk=100))
+
+
+def test_one_token_chunks_equal_decode_bitwise():
+    w = W.decode_workload("one", [5, 200, 700, 1500], num_q_heads=32, num_kv_heads=8,
+                          head_dim=128, dtype="bf16", seed=9)
+    w.q_start = np.arange(5, dtype=np.int32)
+    d = DeviceStep(w)
+    d.cache_ops()
+    a = d.decode().clone()
+    b = d.prefill(torch.empty_like(a))
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_bad_query_ranges_are_counted_and_skipped():
+    w = W.chunk_workload("bad", [50, 60, 70], [5, 6, 7], num_q_heads=4, num_kv_heads=4,
+                         head_dim=64, dtype="f16", seed=4)
+    d = DeviceStep(w)
+    d.cache_ops()
+    qs = torch.from_numpy(w.q_start).cuda()
+    qs[2] = 100                         # sequence 1's range runs past the q rows: skipped
+    d.out.fill_(5.0)
+    pa.prefill_chunk(d.out, d.q, qs, d.k_cache, d.v_cache, d.bt, d.cl, scale=w.scale,
+                     max_query_len=7, max_context_len=70, partition_tokens=512,
+                     dev_error=d.err)
+    torch.cuda.synchronize()
+    assert int(d.err.item()) >= 1
+    kc, vc = oracle_caches_after_step(w)
+    ref = oracle.prefill_chunk(w.q, w.q_start, kc, vc, w.block_tables, w.context_lens, w.scale,
+                               w.dtype)
+    out = to_f64(d.out)
+    assert_decode_close(out[:5], ref[:5])          # sequence 0 is intact
+    assert (out[5:11] == 5.0).all()                # sequence 1 was skipped, nothing written
