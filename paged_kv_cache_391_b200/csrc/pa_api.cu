@@ -67,6 +67,28 @@ pa_status encode_pool_map(CUtensorMap* map, const void* pool, int64_t num_blocks
   return PA_OK;
 }
 
+// q [tokens][H_q][D] as a 3-D tensor (D innermost); a box is 64 columns x the
+// `group` heads of one KV head x 128 / group tokens = 128 rows of 128 bytes,
+// 128-byte swizzled: one K-major operand chunk of a 128-row query tile.
+pa_status encode_query_map(CUtensorMap* map, const void* q, int32_t num_q_tokens,
+                           int32_t num_q_heads, int32_t head_dim, int32_t group, pa_dtype dtype) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return driver_fail("cuTensorMapEncodeTiled lookup", -1);
+  const cuuint64_t row = (cuuint64_t)head_dim * 2;
+  cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)num_q_tokens};
+  cuuint64_t strides[2] = {row, row * num_q_heads};
+  cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map,
+                      dtype == PA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                      3, const_cast<void*>(q), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return driver_fail("cuTensorMapEncodeTiled (query)", (int)r);
+  return PA_OK;
+}
+
 int64_t max_partitions(int32_t max_context_len, int32_t partition_tokens) {
   if (partition_tokens <= 0 || max_context_len <= partition_tokens) return 1;
   return ((int64_t)max_context_len + partition_tokens - 1) / partition_tokens;
@@ -226,6 +248,16 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   a.max_parts = (int32_t)parts;
   a.dev_error = dev_error;
   a.bf16 = dtype == PA_DTYPE_BF16;
+  // Long query chunks (at least 64 rows of (token, head) per KV head) are a
+  // dense contraction: run them on the tcgen05 tensor cores.
+  if (q_start && (int64_t)max_query_len * group_size >= 64 && pa::prefill_tc_supported(a)) {
+    CUtensorMap tm_q;
+    st = encode_query_map(&tm_q, q, num_q_tokens, num_q_heads, head_dim, group_size, dtype);
+    if (st != PA_OK) return st;
+    cudaError_t e = pa::launch_prefill_tc(a, tm_q, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = pa::launch_reduce(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : cuda_fail(e);
+  }
   cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }

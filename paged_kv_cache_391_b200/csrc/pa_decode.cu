@@ -602,6 +602,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   }
 }
 
+template <typename T, int D>
+static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t stream);
+
 template <typename T, int D, bool kTwoRows, bool kMulti>
 static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
   using SM = DecodeSmem<D>;
@@ -615,7 +618,14 @@ static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
       a.num_q_heads, a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
       a.max_parts, a.dev_error);
   e = cudaGetLastError();
-  if (e != cudaSuccess || a.max_parts <= 1) return e;
+  if (e != cudaSuccess) return e;
+  return launch_reduce_typed<T, D>(a, stream);
+}
+
+template <typename T, int D>
+static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t stream) {
+  cudaError_t e = cudaSuccess;
+  if (a.max_parts <= 1) return e;
   const int rows = a.num_q_tokens * a.num_q_heads;
   if (a.max_parts > kWarpRowMaxParts) {
     const size_t wbytes = (size_t)a.max_parts * sizeof(float);
@@ -650,6 +660,14 @@ static cudaError_t launch_dtype(const DecodeLaunch& a, cudaStream_t stream) {
                : launch_typed<T, 128, false, false>(a, stream);
   return two ? launch_typed<T, 64, true, false>(a, stream)
              : launch_typed<T, 64, false, false>(a, stream);
+}
+
+cudaError_t launch_reduce(const DecodeLaunch& a, cudaStream_t stream) {
+  if (a.bf16)
+    return a.head_dim == 128 ? launch_reduce_typed<__nv_bfloat16, 128>(a, stream)
+                             : launch_reduce_typed<__nv_bfloat16, 64>(a, stream);
+  return a.head_dim == 128 ? launch_reduce_typed<__half, 128>(a, stream)
+                           : launch_reduce_typed<__half, 64>(a, stream);
 }
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {

@@ -117,6 +117,7 @@ struct Elem;
 
 template <>
 struct Elem<__half> {
+  static constexpr bool kBf16 = false;
   static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
     asm volatile(
@@ -137,6 +138,7 @@ struct Elem<__half> {
 
 template <>
 struct Elem<__nv_bfloat16> {
+  static constexpr bool kBf16 = true;
   static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
     asm volatile(

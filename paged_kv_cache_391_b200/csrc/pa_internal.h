@@ -42,6 +42,15 @@ struct DecodeLaunch {
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 
+// The log-sum-exp reduce of split partitions alone (no-op for one partition).
+cudaError_t launch_reduce(const DecodeLaunch& a, cudaStream_t stream);
+
+// Query chunks on the tcgen05 tensor cores: supported shapes, and the launch
+// (partition kernel; the caller runs launch_reduce after it). tm_q maps q as
+// [tokens][H_q][D] with boxes of 64 columns x group heads x 128/group tokens.
+bool prefill_tc_supported(const DecodeLaunch& a);
+cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q, cudaStream_t stream);
+
 // Records a CUDA error for pa_last_cuda_error() and returns PA_ERR_CUDA.
 pa_status record_cuda_error(cudaError_t e);
 
