@@ -10,19 +10,22 @@
 //
 // One CTA per (128-row query tile, partition, KV head, sequence); tile rows are
 // (query token, head) pairs of the KV head's query group. 160 threads:
-//  * warps 0-3: softmax. Thread r owns row r: TMEM lane r of S and O.
+//  * warps 0-3: softmax. Thread r owns row r: TMEM lane r of S, P and O.
 //  * warp 4, one lane: producer. It issues every TMA load (Q once; per step
-//    K and V of 4 cache blocks = 64 keys into a 2-stage ring) and every MMA:
-//      S[j%2] = Q K_j^T        (M=128, N=64, K=D; both operands K-major)
-//      O     += P_j V_j        (M=128, N=D, K=64; P K-major, V MN-major)
+//    K and V of 4 cache blocks = 64 keys, each in its own 2-stage ring) and
+//    every MMA:
+//      S[j%2] = Q K_j^T   (M=128, N=64, K=D; Q and K K-major in shared memory)
+//      O     += P_j V_j   (M=128, N=D, K=64; P K-major, V MN-major)
 //    S is double-buffered in TMEM so S(j+1) runs while the softmax of step j
-//    does. P_j (bf16) is written by the softmax warps into the shared memory
-//    of K_j, which S(j) no longer needs.
-// Online softmax per row in fp32, base 2; O is rescaled in TMEM when a row's
-// maximum grows. Keys past the context, past the row's causal limit, or in a
-// block with a bad table entry are masked to -inf, and V rows past the context
-// are zeroed before P.V (0 * stale data must stay 0). All waits are bounded;
-// TMEM is released on every path.
+//    does; the softmax writes P_j (bf16, 128-byte swizzled) into one shared
+//    buffer once P.V(j-1) has read P_{j-1}. K_j's stage is refilled as soon as
+//    S(j) is done, V_j's once P.V(j) is, so S(j+2) never waits for P.V(j).
+// Online softmax per row in fp32, base 2 (hardware ex2); a row's reference
+// maximum and O are only rescaled when the maximum grows by more than 2^8.
+// Keys past the context, past the row's causal limit, or in a block with a bad
+// table entry are masked to -inf, and V rows past the context are zeroed
+// before P.V (0 * stale data must stay 0). All waits are bounded; TMEM is
+// released on every path.
 #include <math.h>
 
 #include <type_traits>
@@ -46,22 +49,34 @@ constexpr uint32_t kTmemCols = 256;        // S0 [0,64) S1 [64,128) O [128,256)
 constexpr uint32_t kOCol = 128;
 
 constexpr int kQBytes = kRows * kD * 2;            // 32 KiB: [chunk][128 rows][128 B]
-constexpr int kKBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]; later P
+constexpr int kKBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]
 constexpr int kVBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]
-constexpr int kStageBytes = kKBytes + kVBytes;
+constexpr int kPBytes = kRows * kKeys * 2;        // 16 KiB: [128 rows][128 B] bf16 P
 constexpr int kQOff = 0;
-constexpr int kStageOff = kQBytes;
-constexpr int kBarOff = kStageOff + 2 * kStageBytes;
-// barriers: q_full, kv_full[2], s_full[2], p_ready, pv_done ; then the TMEM address
-constexpr int kNumBars = 7;
+constexpr int kKOff = kQBytes;                     // K stages 0, 1
+constexpr int kVOff = kKOff + 2 * kKBytes;         // V stages 0, 1
+constexpr int kPOff = kVOff + 2 * kVBytes;
+constexpr int kBarOff = kPOff + kPBytes;
+// barriers: q_full, k_full[2], v_full[2], s_full[2], p_ready, pv_done; then the TMEM address
+constexpr int kNumBars = 9;
 constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kTmemSlotOff + 16;
-constexpr int kSmemAlloc = kSmemBytes + 1024;
-static_assert(kRows * 128 == kKBytes, "P (128 rows x 64 bf16) must fit in a K stage");
+// No alignment slack: two CTAs per SM need all of it. The dynamic shared
+// memory is declared 1024-byte aligned and the kernel checks it.
+constexpr int kSmemAlloc = kSmemBytes;
 
-__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk16) {
-  return row * 128 + ((chunk16 ^ (row & 7)) << 4);
+// 2^x by the hardware approximation (ex2.approx, relative error ~2^-22; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
+
+// A row's running maximum is only moved (and O rescaled) when the new
+// maximum exceeds it by more than 2^8: until then P is taken against the
+// older, smaller reference (values up to 256, exact in the fp32 sums and
+// representable in bf16), and O / l is unchanged by the choice of reference.
+constexpr float kRescaleLog2 = 8.f;
 
 template <typename T>
 __global__ void __launch_bounds__(kThreadsTc)
@@ -75,17 +90,22 @@ __global__ void __launch_bounds__(kThreadsTc)
                       int64_t num_blocks, int max_context_len, float scale_log2,
                       int part_blocks, int max_parts, int32_t* __restrict__ dev_error) {
   using E = Elem<T>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;  // [2]
-  uint64_t* s_full = bars + 3;   // [2]
-  uint64_t* p_ready = bars + 5;
-  uint64_t* pv_done = bars + 6;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* v_full = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;   // [2]
+  uint64_t* p_ready = bars + 7;
+  uint64_t* pv_done = bars + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlotOff);
 
+  if (smem_addr(smem) & 1023) {  // the 128-byte swizzle needs 1024-byte aligned tiles
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && dev_error)
+      atomicAdd(dev_error, 1);
+    return;
+  }
   const int kvh = blockIdx.y, seq = blockIdx.z;
   const int part = (int)(blockIdx.x % (unsigned)max_parts);
   const int qtile = (int)(blockIdx.x / (unsigned)max_parts);
@@ -124,8 +144,10 @@ __global__ void __launch_bounds__(kThreadsTc)
   // ---- set-up: barriers (thread 0), TMEM (warp 0)
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(&kv_full[0], 1);
-    mbar_init(&kv_full[1], 1);
+    mbar_init(&k_full[0], 1);
+    mbar_init(&k_full[1], 1);
+    mbar_init(&v_full[0], 1);
+    mbar_init(&v_full[1], 1);
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
     mbar_init(p_ready, kSoftmaxWarps * 32);
@@ -143,55 +165,95 @@ __global__ void __launch_bounds__(kThreadsTc)
   bool failed = false;
 
   const uint32_t q_s = smem_addr(smem + kQOff);
-  auto stage_k = [&](int st) { return smem + kStageOff + st * kStageBytes; };
-  auto stage_v = [&](int st) { return smem + kStageOff + st * kStageBytes + kKBytes; };
+  auto stage_k = [&](int st) { return smem + kKOff + st * kKBytes; };
+  auto stage_v = [&](int st) { return smem + kVOff + st * kVBytes; };
+  uint8_t* p_buf = smem + kPOff;
   const int32_t* bt_row = block_tables + (size_t)seq * bt_stride;
 
   if (warp == kSoftmaxWarps) {
     // =============================== producer ===============================
-    if (lane == 0) {
+    {
+      // The whole warp runs the producer's control flow (so the block table
+      // can be read 32 entries per coalesced load and broadcast by shuffle);
+      // lane 0 alone issues TMA loads, MMAs and commits.
+      const bool leader = lane == 0;
       const uint32_t id_s = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kKeys, false, false);
       const uint32_t id_pv = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kD, false, true);
       // What is in flight, for the drain after a wait that gave up.
-      int kv_pending[2] = {-1, -1};     // step whose K/V load into the stage is unconfirmed
-      uint64_t* last_bar = nullptr;     // barrier of the last MMA commit, and its parity
+      int k_pending[2] = {-1, -1}, v_pending[2] = {-1, -1};
+      uint64_t* last_bar = nullptr;  // barrier of the last MMA commit, and its parity
       uint32_t last_parity = 0;
-      auto load_kv = [&](int j) {
+      // Physical ids of the partition's blocks, 32 per register window: lane i
+      // holds entry 32 * win + i (-1 past the keys or for a bad entry).
+      const int lb_first = key_begin / 16;
+      const int nblk_keys = (key_end - key_begin + 15) / 16;
+      auto load_window = [&](int w) {
+        const int i = 32 * w + lane;
+        int p = -1;
+        if (i < nblk_keys) {
+          p = __ldg(bt_row + lb_first + i);
+          if (p < 0 || p >= num_blocks) p = -1;
+        }
+        return p;
+      };
+      int win = 0, pid_cur = load_window(0), pid_nxt = load_window(1);
+      auto pid_of = [&](int i) {  // all lanes; i within the current or the next window
+        const int v = (i >> 5) == win ? pid_cur : pid_nxt;
+        return __shfl_sync(0xffffffffu, v, i & 31);
+      };
+      // K (or V) of the step's four cache blocks into stage j % 2; blocks past
+      // the keys or with a bad table entry are not loaded.
+      auto load = [&](int j, bool is_v) {
         const int st = j & 1;
-        kv_pending[st] = j;
-        uint32_t bytes = 0;
-        const int lb0 = key_begin / 16 + j * kStepBlocks;
+        uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
+        (is_v ? v_pending : k_pending)[st] = j;
+        uint8_t* dst = is_v ? stage_v(st) : stage_k(st);
+        const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+        while (((j * kStepBlocks) >> 5) > win) {  // a step's 4 entries share one window
+          ++win;                       // slide the table window forward
+          pid_cur = pid_nxt;
+          pid_nxt = load_window(win + 1);
+        }
         int pids[kStepBlocks];
+        uint32_t bytes = 0;
 #pragma unroll
         for (int b = 0; b < kStepBlocks; ++b) {
-          const int lb = lb0 + b;
-          int p = -1;
-          if (lb * 16 < key_end) {
-            p = __ldg(bt_row + lb);
-            if (p < 0 || p >= num_blocks) p = -1;
-          }
-          pids[b] = p;
-          if (p >= 0) bytes += 2 * kChunks * 2048;
+          pids[b] = pid_of(j * kStepBlocks + b);
+          if (pids[b] >= 0) bytes += kChunks * 2048;
         }
+        if (!leader) return;
         if (bytes == 0) {
-          mbar_arrive(&kv_full[st]);
+          mbar_arrive(bar);
           return;
         }
-        mbar_arrive_expect_tx(&kv_full[st], bytes);
+        mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
         for (int b = 0; b < kStepBlocks; ++b) {
           if (pids[b] < 0) continue;
 #pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            tma_load_4d(stage_k(st) + c * (kKeys * 128) + b * 2048, &tm_k, &kv_full[st], c * 64,
-                        0, kvh, pids[b]);
-            tma_load_4d(stage_v(st) + c * (kKeys * 128) + b * 2048, &tm_v, &kv_full[st], c * 64,
-                        0, kvh, pids[b]);
-          }
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_4d(dst + c * (kKeys * 128) + b * 2048, map, bar, c * 64, 0, kvh, pids[b]);
         }
+      };
+      // Every wait is taken by all lanes and agreed on, so the warp stays converged.
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+      };
+      auto wait_k = [&](int j) {
+        const bool ok = wait_all(&k_full[j & 1], (j >> 1) & 1);
+        if (ok) k_pending[j & 1] = -1;
+        return ok;
+      };
+      auto wait_v = [&](int j) {
+        const bool ok = wait_all(&v_full[j & 1], (j >> 1) & 1);
+        if (ok) v_pending[j & 1] = -1;
+        return ok;
       };
       auto issue_s = [&](int j) {
         const int st = j & 1;
+        last_bar = &s_full[st];
+        last_parity = (uint32_t)((j >> 1) & 1);
+        if (!leader) return;
         const uint32_t k_s = smem_addr(stage_k(st));
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -201,13 +263,14 @@ __global__ void __launch_bounds__(kThreadsTc)
           tc::mma_f16(tmem + (uint32_t)(st * kKeys), a, b, id_s, kk > 0);
         }
         tc::commit(&s_full[st]);
-        last_bar = &s_full[st];
-        last_parity = (uint32_t)((j >> 1) & 1);
       };
       auto issue_pv = [&](int j) {
         const int st = j & 1;
-        const uint32_t p_s = smem_addr(stage_k(st));
+        last_bar = pv_done;
+        last_parity = (uint32_t)(j & 1);
+        if (!leader) return;
         const uint32_t v_s = smem_addr(stage_v(st));
+        const uint32_t p_s = smem_addr(p_buf);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           const uint64_t a = tc::smem_desc_sw128(p_s + kk * 32, 16, 1024);
@@ -215,51 +278,57 @@ __global__ void __launch_bounds__(kThreadsTc)
           tc::mma_f16(tmem + kOCol, a, b, id_pv, j > 0 || kk > 0);
         }
         tc::commit(pv_done);
-        last_bar = pv_done;
-        last_parity = (uint32_t)(j & 1);
-      };
-      auto wait_kv = [&](int j) {
-        const bool ok = mbar_wait(&kv_full[j & 1], (j >> 1) & 1);
-        if (ok) kv_pending[j & 1] = -1;
-        return ok;
       };
 
-      tma_prefetch_desc(&tm_q);
+      if (leader) tma_prefetch_desc(&tm_q);
       if (n_steps > 0) {
-        mbar_arrive_expect_tx(q_full, kQBytes);
+        if (leader) {
+          mbar_arrive_expect_tx(q_full, kQBytes);
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c)
-          tc::tma_load_3d(smem + kQOff + c * (kRows * 128), &tm_q, q_full, c * 64, q_head0,
-                          q0 + t0);
-        load_kv(0);
-        if (n_steps > 1) load_kv(1);
-        failed = !mbar_wait(q_full, 0) || !wait_kv(0);
-        if (!failed) {
-          tc::fence_after_sync();
-          issue_s(0);
+          for (int c = 0; c < kChunks; ++c)
+            tc::tma_load_3d(smem + kQOff + c * (kRows * 128), &tm_q, q_full, c * 64, q_head0,
+                            q0 + t0);
         }
+        load(0, false);
+        load(0, true);
+        if (n_steps > 1) {
+          load(1, false);
+          load(1, true);
+        }
+        failed = !wait_all(q_full, 0) || !wait_k(0);
+        if (!failed) issue_s(0);
       }
       for (int j = 0; j < n_steps && !failed; ++j) {
+        // S(j+1): its TMEM buffer was read by softmax(j-1), whose p_ready was
+        // awaited in the previous iteration.
         if (j + 1 < n_steps) {
-          if (!wait_kv(j + 1)) { failed = true; break; }
+          if (!wait_k(j + 1)) { failed = true; break; }
           issue_s(j + 1);
         }
-        if (!mbar_wait(p_ready, j & 1)) { failed = true; break; }
+        // V(j+1) into the stage PV(j-1) has finished reading
+        if (j >= 1 && j + 1 < n_steps) {
+          if (!wait_all(pv_done, (j - 1) & 1)) { failed = true; break; }
+          load(j + 1, true);
+        }
+        // K(j+2) into the stage S(j) has finished reading
+        if (j + 2 < n_steps) {
+          if (!wait_all(&s_full[j & 1], (j >> 1) & 1)) { failed = true; break; }
+          load(j + 2, false);
+        }
+        if (!wait_all(p_ready, j & 1) || !wait_v(j)) { failed = true; break; }
         tc::fence_after_sync();
         issue_pv(j);
-        if (j + 2 < n_steps) {
-          if (!mbar_wait(pv_done, j & 1)) { failed = true; break; }
-          load_kv(j + 2);
-        }
       }
       if (failed) {
         // Let the copies and MMAs already issued finish (each wait bounded)
         // before shared memory and TMEM are released.
         (void)mbar_wait(q_full, 0);
-        for (int st = 0; st < 2; ++st)
-          if (kv_pending[st] >= 0) (void)mbar_wait(&kv_full[st], (kv_pending[st] >> 1) & 1);
+        for (int st = 0; st < 2; ++st) {
+          if (k_pending[st] >= 0) (void)mbar_wait(&k_full[st], (k_pending[st] >> 1) & 1);
+          if (v_pending[st] >= 0) (void)mbar_wait(&v_full[st], (v_pending[st] >> 1) & 1);
+        }
         if (last_bar) (void)mbar_wait(last_bar, last_parity);
-        if (dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
+        if (leader && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
       }
     }
   } else {
@@ -269,20 +338,30 @@ __global__ void __launch_bounds__(kThreadsTc)
     const int t = t0 + r / group, h = r % group;         // query token in the chunk, head
     const bool row_ok = t < Tq;
     const int lim = L - Tq + (row_ok ? t : 0);           // last key this row may see
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;                        // reference maximum (log2 units)
+    // keys every row of the tile may see: up to the first row's causal limit
+    const int key_all = min(key_end, L - Tq + t0 + 1);
+    // Validity of the table entries of a step (a bit per cache block), loaded
+    // one step ahead so the table reads never wait in the loop.
+    auto bad_blocks = [&](int j) {
+      int mask = 0;
+      const int lb0 = (key_begin + j * kKeys) / 16;
+#pragma unroll
+      for (int b = 0; b < kStepBlocks; ++b) {
+        const int lb = lb0 + b;
+        if (lb * 16 < key_end) {
+          const int p = __ldg(bt_row + lb);
+          if (p < 0 || p >= num_blocks) mask |= 1 << b;
+        }
+      }
+      return mask;
+    };
+    int bad_next = n_steps > 0 ? bad_blocks(0) : 0;
     for (int j = 0; j < n_steps; ++j) {
       const int st = j & 1;
       const int kb = key_begin + j * kKeys;
-      // table entries of this step (validity only)
-      int bad_mask = 0;
-#pragma unroll
-      for (int b = 0; b < kStepBlocks; ++b) {
-        const int lb = kb / 16 + b;
-        if (lb * 16 < key_end) {
-          const int p = __ldg(bt_row + lb);
-          if (p < 0 || p >= num_blocks) bad_mask |= 1 << b;
-        }
-      }
+      const int bad_mask = bad_next;
+      if (j + 1 < n_steps) bad_next = bad_blocks(j + 1);
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) { failed = true; break; }
       tc::fence_after_sync();
       float s[64];
@@ -297,49 +376,57 @@ __global__ void __launch_bounds__(kThreadsTc)
           s[32 + i] = b2[i];
         }
       }
-      float mx = -INFINITY;
+      // Logits in log2 units are s * scale_log2. Steps wholly inside the
+      // tile's causal horizon need no mask (scale folded into the exp's FMA);
+      // otherwise scale first and give masked keys -inf.
+      const bool need_mask = kb + kKeys > key_all || bad_mask != 0;
+      float mx, cc;
+      if (need_mask) {
+        mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int kp = kb + i;
-        const bool ok = kp < key_end && kp <= lim && !((bad_mask >> (i >> 4)) & 1);
-        s[i] = ok ? s[i] * scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 64; ++i) {
+          const int kp = kb + i;
+          const bool ok = kp < key_end && kp <= lim && !((bad_mask >> (i >> 4)) & 1);
+          s[i] = ok ? s[i] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, s[i]);
+        }
+        cc = 1.f;
+      } else {
+        float hi = s[0], lo = s[0];
+#pragma unroll
+        for (int i = 1; i < 64; ++i) {
+          hi = fmaxf(hi, s[i]);
+          lo = fminf(lo, s[i]);
+        }
+        mx = (scale_log2 >= 0.f ? hi : lo) * scale_log2;
+        cc = scale_log2;
       }
-      const float m_new = fmaxf(m, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = exp2f(m - m_use);
+      float alpha = 1.f;
+      if (mx > m + kRescaleLog2 || m == -INFINITY) {
+        const float m_new = fmaxf(m, mx);
+        alpha = m == -INFINITY ? 0.f : fast_exp2(m - m_new);
+        m = m_new;
+      }
+      const float m_use = m == -INFINITY ? 0.f : m;
       uint32_t pk[32];
       float psum = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        pk[i] = E::pack(exp2f(s[2 * i] - m_use), exp2f(s[2 * i + 1] - m_use));
-        const float2 u = E::unpack(pk[i]);
-        psum += u.x + u.y;
+        const float p0 = fast_exp2(fmaf(s[2 * i], cc, -m_use));
+        const float p1 = fast_exp2(fmaf(s[2 * i + 1], cc, -m_use));
+        psum += p0 + p1;
+        pk[i] = E::pack(p0, p1);
       }
       l = l * alpha + psum;
-      m = m_new;
-      // PV(j-1) must be done: it read the P buffer this step reuses' twin and
-      // writes O, which may be rescaled below.
+      // PV(j-1) must be done before O is rescaled (it writes O).
       if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) { failed = true; break; }
       tc::fence_after_sync();
-      // P row r: 64 bf16 = 128 bytes, 128-byte swizzle, in K_j's shared memory
-      uint8_t* p_row = stage_k(st);
+      // P_j row r: 64 bf16 = 128 bytes, 128-byte swizzle (PV(j-1) has read P_{j-1})
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(p_row + swz(r, c)) =
+        *reinterpret_cast<uint4*>(p_buf + r * 128 + ((c ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      // V rows of keys past the context (the final step only) become zero
-      if (kb + kKeys > key_end || bad_mask) {
-        uint8_t* v = stage_v(st);
-        for (int i = r; i < kKeys * kChunks * 8; i += kSoftmaxWarps * 32) {
-          const int c = i / (kKeys * 8), rem = i % (kKeys * 8);
-          const int key = rem / 8;
-          if (kb + key >= key_end || ((bad_mask >> (key >> 4)) & 1))
-            *reinterpret_cast<uint4*>(v + c * (kKeys * 128) + key * 128 + (rem % 8) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      // rescale O when this row's maximum grew (warp-uniform decision)
+      // rescale O when a row's reference maximum moved (warp-uniform decision)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {
@@ -350,9 +437,21 @@ __global__ void __launch_bounds__(kThreadsTc)
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
           tc::tmem_st32(lane_addr + kOCol + c * 32, o);
         }
-        tc::tmem_wait_st();
       }
-      fence_proxy_async_smem();   // P and zeroed V rows -> visible to the tensor core
+      if (j > 0) tc::tmem_wait_st();
+      // V rows of keys past the context or of bad blocks become zero (once V_j landed)
+      if (kb + kKeys > key_end || bad_mask) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (j >> 1) & 1))) { failed = true; break; }
+        uint8_t* v = stage_v(st);
+        for (int i = r; i < kKeys * kChunks * 8; i += kSoftmaxWarps * 32) {
+          const int c = i / (kKeys * 8), rem = i % (kKeys * 8);
+          const int key = rem / 8;
+          if (kb + key >= key_end || ((bad_mask >> (key >> 4)) & 1))
+            *reinterpret_cast<uint4*>(v + c * (kKeys * 128) + key * 128 + (rem % 8) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();  // P (and zeroed V rows) -> visible to the tensor core
       tc::fence_before_sync();
       mbar_arrive(p_ready);
     }

@@ -291,8 +291,10 @@ def chunked_prefill(seed: int = 397, batch: int = 16, chunk: int = 256) -> Decod
     prefix already cached."""
     rng = np.random.default_rng(seed)
     lens = rng.integers(1024, 8192, size=batch, endpoint=True)
+    # 16 sequences x 8 KV heads x 8 query tiles already fill the GPU: no split-K
     return chunk_workload("chunked_prefill", lens, np.full(batch, chunk), num_q_heads=32,
-                          num_kv_heads=8, head_dim=128, dtype="bf16", seed=seed, rng=rng)
+                          num_kv_heads=8, head_dim=128, dtype="bf16", seed=seed, rng=rng,
+                          partition_tokens=0)
 
 
 # ---------------------------------------------------------------------------

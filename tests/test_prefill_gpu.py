@@ -83,3 +83,14 @@ def test_bad_query_ranges_are_counted_and_skipped():
     out = to_f64(d.out)
     assert_decode_close(out[:5], ref[:5])          # sequence 0 is intact
     assert (out[5:11] == 5.0).all()                # sequence 1 was skipped, nothing written
+
+
+@pytest.mark.parametrize("scale", [0.0, 1.0])
+def test_tensor_core_chunks_scale_zero_and_large_logits(scale):
+    """On the tcgen05 path (D 128, many rows): scale 0 makes every row the
+    mean of the values it may see; scale 1 with q and K of norm ~11 gives
+    logits of tens to hundreds, so the running maximum moves a lot."""
+    w = W.chunk_workload("s", [900, 333], [200, 96], num_q_heads=8, num_kv_heads=2,
+                         head_dim=128, dtype="bf16", seed=int(scale) + 40)
+    w.scale = scale
+    _check(w)
