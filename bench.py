@@ -7,7 +7,8 @@ this step's tokens, and paged decode attention (partition kernel plus the
 log-sum-exp reduce when a context spans several partitions), all through
 libpa's C ABI on the current CUDA stream.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|shared_prefix|long|tiny]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|shared_prefix|long|...]
+                  [--scheduler grid|persistent]
   python bench.py --impl reference ...   # the fp64 CPU oracle, timed on the host cores
 
 Multi-GPU (launched by torch.distributed.run): every rank runs its own
@@ -48,6 +49,9 @@ WORKLOAD_TEXT = {
                    "(causal in the chunk), H_q=32, H_kv=8, D=128, bf16, ctx lognormal(1024, 1)",
     "chunked_prefill": "chunked prefill, Llama-3-8B shape: 16 prompts of U[1024,8192] tokens, "
                        "next 256-token chunk each, H_q=32, H_kv=8, D=128, bf16",
+    "skewed": "skewed-length decode, Llama-3-8B GQA shape: batch 256, 4 contexts U[65536,131072] "
+              "among 252 lognormal(median 512, sigma 0.7) clipped [16,4096], H_q=32, H_kv=8, "
+              "D=128, bf16",
 }
 
 
@@ -63,6 +67,9 @@ def parse():
                     help="step: the decode step (default); swap: preemption swap-out/in; "
                          "blockmgr: host block-manager throughput (no GPU)")
     ap.add_argument("--partition-tokens", type=int, default=None)
+    ap.add_argument("--scheduler", default="grid", choices=["grid", "persistent"],
+                    help="decode schedule: grid = pa_decode (one CTA per partition); "
+                         "persistent = pa_decode_persistent (plan + work queue)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -95,17 +102,18 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, batch):
+def recorded_traffic(workload: str, batch, scheduler: str = "grid"):
     """DRAM bytes (read + write) per pa_decode call from the ncu capture
     recorded in profiles/dram_traffic.txt for this workload, or None when
     there is none or the kernel sources changed since it was taken."""
     if batch is not None or not os.path.exists(TRAFFIC_FILE):
         return None
     want = kernel_source_hash()
+    key = workload if scheduler == "grid" else f"{workload}:{scheduler}"
     with open(TRAFFIC_FILE) as f:
         for line in f:
             parts = line.split("#")[0].split()
-            if len(parts) >= 3 and parts[0] == workload and parts[1] == want:
+            if len(parts) >= 3 and parts[0] == key and parts[1] == want:
                 return int(parts[2])
     return None
 
@@ -317,14 +325,16 @@ def run_gpu(args, rank, world, device):
     out = torch.empty(w.q.shape, dtype=dt, device=device)
     P = w.partition_tokens
     n_q = int(w.q.shape[0])
-    ws = pa.alloc_workspace(n_q, w.num_q_heads, w.head_dim, w.max_context_len, P, device)
+    persistent = args.scheduler == "persistent" and w.q_start is None
+    ws = pa.alloc_workspace(n_q, w.num_q_heads, w.head_dim, w.max_context_len, P, device,
+                            persistent=persistent)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
     max_ctx = w.max_context_len
     max_q = int(np.diff(w.q_start).max()) if w.q_start is not None else 1
     max_parts = 1 if (P == 0 or max_ctx <= P) else -(-max_ctx // P)
     launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + \
-        1 + (1 if max_parts > 1 else 0)
+        1 + (1 if max_parts > 1 else 0) + (1 if persistent else 0)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
@@ -342,7 +352,7 @@ def run_gpu(args, rank, world, device):
         else:
             pa.decode(o, x["q"], k_cache, v_cache, x["bt"], x["cl"], scale=w.scale,
                       max_context_len=max_ctx, partition_tokens=P, workspace=ws, dev_error=err,
-                      stream=stream)
+                      stream=stream, persistent=persistent)
         if e_dec is not None:
             e_dec[1].record(stream)
 
@@ -622,6 +632,9 @@ def main():
             "mean_context_len": float(np.mean(w.context_lens)),
             "kv_bytes_per_step": kv_bytes,
             "step": "copy_blocks (if forks) + write_kv + decode (partitions + LSE reduce)",
+            "scheduler": ("persistent: plan kernel + work-queue grid of SMs x resident CTAs"
+                          if args.scheduler == "persistent" and w.q_start is None
+                          else "grid: one CTA per (partition, KV head, sequence)"),
             "accumulate": "fp32",
             "l2": l2_note(w),
             "parallelism": f"dp{world} (independent sequences per GPU)",
@@ -629,8 +642,13 @@ def main():
         "seq_steps_per_s": round(seqs_total * K / (elapsed_ms / 1e3), 1),
         "hbm_frac_of_peak": round(value / peak, 4),
         "roofline": {
-            "kernel": ("pa_prefill_chunk" if w.q_start is not None else "pa_decode") +
-                      " (decode_partition_kernel + lse_reduce_kernel)",
+            "kernel": (("pa_prefill_chunk (prefill_tc_kernel on tcgen05 + lse_reduce_kernel)"
+                        if int(np.diff(w.q_start).max()) * w.group_size >= 64 else
+                        "pa_prefill_chunk (decode_partition_kernel + lse_reduce_kernel)")
+                       if w.q_start is not None else
+                       "pa_decode_persistent (decode_plan_kernel + decode_persistent_kernel + "
+                       "lse_reduce_kernel)" if args.scheduler == "persistent" else
+                       "pa_decode (decode_partition_kernel + lse_reduce_kernel)"),
             "bound": "tensor" if tensor_bound else "hbm",
             "achieved": round(flops / (dec_ms / 1e3) / 1e12, 2) if tensor_bound
             else round(dec_achieved, 1),
@@ -643,7 +661,7 @@ def main():
             "tflops": round(flops / (dec_ms / 1e3) / 1e12, 2),
             "flops_per_launch": flops,
             "algorithmic_bytes_per_launch": sb["decode"],
-            "traffic": recorded_traffic(args.workload, args.batch),
+            "traffic": recorded_traffic(args.workload, args.batch, args.scheduler),
             "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
                             "decode_partition_kernel + lse_reduce per call "
                             "(profiles/dram_traffic.txt; null if the kernel changed since)",

@@ -134,6 +134,41 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     int32_t* dev_error, pa_dtype dtype, void* stream);
 
 /*
+ * Bytes of workspace pa_decode_persistent needs: pa_decode's partials (if
+ * any), a work list of num_seqs * partitions 32-bit items, and 256 bytes of
+ * plan state. Never 0 for num_seqs > 0.
+ */
+size_t pa_decode_persistent_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                           int32_t head_dim, int32_t max_context_len,
+                                           int32_t partition_tokens);
+
+/*
+ * pa_decode scheduled as a work queue ("New Developments in 2026": PersistentKV
+ * organises decode by pages, KV-head groups, sequence splits and work queues).
+ * Same arguments, same result bit for bit as pa_decode with the same
+ * partition_tokens: each (sequence, partition, KV head) item is computed the
+ * same way; only which CTA computes it, and when, differ. A plan kernel lists
+ * the sequences' non-empty partitions on the device, longest first (so the
+ * host needs no copy of context_lens); one wave of CTAs (SMs x resident CTAs
+ * per SM) then pulls (item, KV head) pairs from a counter until none are
+ * left. On skewed context lengths this removes the empty CTAs a grid sized by
+ * max_context_len launches and the tail of a long item started last.
+ *   workspace  device, >= pa_decode_persistent_workspace_size(...) bytes,
+ *              256-byte aligned; never NULL. It holds the plan between the
+ *              kernels of one call, so concurrent calls need separate ones.
+ * Errors: as pa_decode; PA_ERR_UNSUPPORTED also when a sequence may have more
+ * than 65536 partitions or num_seqs * partitions * KV heads exceeds 2^31 - 1.
+ */
+pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               int32_t block_table_stride, const int32_t* context_lens,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t group_size,
+                               int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                               int32_t max_context_len, float scale, int32_t partition_tokens,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                               pa_dtype dtype, void* stream);
+
+/*
  * Attention of several query tokens per sequence over the paged cache, causal
  * within the chunk: the query tokens of sequence s are q rows q_start[s] ..
  * q_start[s+1]-1 and are the LAST Tq = q_start[s+1] - q_start[s] tokens of its

@@ -168,6 +168,16 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
   return round256(rows * head_dim * sizeof(float)) + round256(rows * sizeof(float));
 }
 
+size_t pa_decode_persistent_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                           int32_t head_dim, int32_t max_context_len,
+                                           int32_t partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const int64_t parts = max_partitions(max_context_len, partition_tokens);
+  return pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                  partition_tokens) +
+         round256((size_t)num_seqs * parts * sizeof(uint32_t)) + 256;
+}
+
 }  // extern "C"
 
 namespace {
@@ -182,7 +192,7 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
                     int32_t group_size, int32_t head_dim, int32_t block_size,
                     int64_t num_blocks, int32_t max_context_len, float scale,
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
-                    int32_t* dev_error, pa_dtype dtype, void* stream) {
+                    int32_t* dev_error, pa_dtype dtype, void* stream, bool persistent = false) {
   if (num_seqs < 0 || num_q_heads < 1 || group_size < 1 || num_blocks < 1 ||
       max_context_len < 0 || partition_tokens < 0 || !valid_dtype(dtype) || !isfinite(scale) ||
       num_q_tokens < 0 || max_query_len < 0)
@@ -208,11 +218,19 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   const int64_t qtiles = q_start ? ((int64_t)max_query_len * group_size + 15) / 16 : 1;
   if (qtiles < 1) return PA_OK;  // no query token can exist
   if (parts * qtiles > 0x7fffffff) return PA_ERR_UNSUPPORTED;
+  // The work queue packs (sequence, partition) into 16 + 16 bits and counts
+  // (item, KV head) pairs in 32 bits.
+  if (persistent && (parts > 65536 || (int64_t)num_seqs * parts * num_kv_heads > 0x7fffffff))
+    return PA_ERR_UNSUPPORTED;
   const size_t need = pa_decode_workspace_size(num_q_tokens, num_q_heads, head_dim,
                                                max_context_len, partition_tokens);
-  if (need > 0) {
+  const size_t need_all =
+      persistent ? pa_decode_persistent_workspace_size(num_q_tokens, num_q_heads, head_dim,
+                                                       max_context_len, partition_tokens)
+                 : need;
+  if (need_all > 0) {
     if (!workspace || !aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
-    if (workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace_bytes < need_all) return PA_ERR_WORKSPACE_TOO_SMALL;
   }
 
   pa::DecodeLaunch a;
@@ -248,6 +266,15 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   a.max_parts = (int32_t)parts;
   a.dev_error = dev_error;
   a.bf16 = dtype == PA_DTYPE_BF16;
+  a.items = nullptr;
+  a.plan = nullptr;
+  if (persistent) {
+    char* tail = static_cast<char*>(workspace) + need;
+    a.items = reinterpret_cast<uint32_t*>(tail);
+    a.plan = reinterpret_cast<int32_t*>(tail + round256((size_t)num_seqs * parts * sizeof(uint32_t)));
+    cudaError_t e = pa::launch_decode_persistent(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : cuda_fail(e);
+  }
   // Long query chunks (at least 64 rows of (token, head) per KV head) are a
   // dense contraction: run them on the tcgen05 tensor cores.
   if (q_start && (int64_t)max_query_len * group_size >= 64 && pa::prefill_tc_supported(a)) {
@@ -277,6 +304,20 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                    block_table_stride, context_lens, num_seqs, num_q_heads, group_size, head_dim,
                    block_size, num_blocks, max_context_len, scale, partition_tokens, workspace,
                    workspace_bytes, dev_error, dtype, stream);
+}
+
+pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               int32_t block_table_stride, const int32_t* context_lens,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t group_size,
+                               int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                               int32_t max_context_len, float scale, int32_t partition_tokens,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                               pa_dtype dtype, void* stream) {
+  return attention(out, q, nullptr, num_seqs, 1, k_cache, v_cache, block_tables,
+                   block_table_stride, context_lens, num_seqs, num_q_heads, group_size, head_dim,
+                   block_size, num_blocks, max_context_len, scale, partition_tokens, workspace,
+                   workspace_bytes, dev_error, dtype, stream, true);
 }
 
 pa_status pa_prefill_chunk(void* out, const void* q, const int32_t* q_start,

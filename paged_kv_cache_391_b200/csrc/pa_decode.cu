@@ -74,32 +74,62 @@ __device__ __forceinline__ uint32_t tile_off(int t, int d) {
   return (uint32_t)((d >> 6) * 2048 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4) + (d & 7) * 2);
 }
 
+// The arguments every work item shares.
+template <typename T>
+struct ItemArgs {
+  const CUtensorMap* tm_k;
+  const CUtensorMap* tm_v;
+  T* out;
+  float* part_o;
+  float* part_lse;
+  const T* q;
+  const int32_t* q_start;
+  int num_q_tokens, max_query_len;
+  const int32_t* block_tables;
+  int bt_stride;
+  const int32_t* context_lens;
+  int num_q_heads, group;
+  int64_t num_blocks;
+  int max_context_len;
+  float scale_log2;
+  int part_blocks, max_parts;
+  int32_t* dev_error;
+};
+
+// One work item: (partition, KV head, sequence, query tile), by the whole CTA.
 // kMulti = false: one query token per sequence (decode); the tile's rows are
 // the query heads of one KV head. kMulti = true: each sequence's last Tq
 // context tokens are queries (a prompt chunk, or speculative draft tokens);
 // the tile's rows are (query token, head) pairs, 16 per tile, and query token
 // t sees the context up to its own position L - Tq + t (causal in the chunk).
+// `ring` counts the tiles this warp has consumed from its ring before the
+// item (stage and mbarrier parity continue from it across items); with
+// init_bars the warp first initialises its ring's barriers. Returns true if a
+// tile wait ran out of time (the error is counted in dev_error).
 template <typename T, int D, bool kTwoRows, bool kMulti>
-__global__ void __launch_bounds__(kThreads)
-    decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, T* __restrict__ out,
-                            float* __restrict__ part_o, float* __restrict__ part_lse,
-                            const T* __restrict__ q, const int32_t* __restrict__ q_start,
-                            int num_q_tokens, int max_query_len,
-                            const int32_t* __restrict__ block_tables, int bt_stride,
-                            const int32_t* __restrict__ context_lens, int num_q_heads, int group,
-                            int64_t num_blocks, int max_context_len, float scale_log2,
-                            int part_blocks, int max_parts, int32_t* __restrict__ dev_error) {
+__device__ __forceinline__ bool attend_item(const ItemArgs<T>& A, uint8_t* smem, uint64_t* bars,
+                                            int part, int kvh, int seq, int qtile,
+                                            bool init_bars, uint32_t& ring) {
   using SM = DecodeSmem<D>;
   using E = Elem<T>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOffset);
+  const CUtensorMap* tm_k = A.tm_k;
+  const CUtensorMap* tm_v = A.tm_v;
+  T* __restrict__ out = A.out;
+  float* __restrict__ part_o = A.part_o;
+  float* __restrict__ part_lse = A.part_lse;
+  const T* __restrict__ q = A.q;
+  const int32_t* __restrict__ q_start = A.q_start;
+  const int num_q_tokens = A.num_q_tokens, max_query_len = A.max_query_len;
+  const int32_t* __restrict__ block_tables = A.block_tables;
+  const int bt_stride = A.bt_stride;
+  const int32_t* __restrict__ context_lens = A.context_lens;
+  const int num_q_heads = A.num_q_heads, group = A.group;
+  const int64_t num_blocks = A.num_blocks;
+  const int max_context_len = A.max_context_len;
+  const float scale_log2 = A.scale_log2;
+  const int part_blocks = A.part_blocks, max_parts = A.max_parts;
+  int32_t* __restrict__ dev_error = A.dev_error;
 
-  const int kvh = blockIdx.y, seq = blockIdx.z;
-  const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x;
-  const int qtile = kMulti ? (int)(blockIdx.x / (unsigned)max_parts) : 0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const bool counter = part == 0 && kvh == 0 && qtile == 0 && tid == 0 && dev_error;
@@ -116,7 +146,7 @@ __global__ void __launch_bounds__(kThreads)
     Tq = q_start[seq + 1] - q0;
     if (q0 < 0 || Tq < 0 || q0 + Tq > num_q_tokens) {
       if (counter) atomicAdd(dev_error, 1);  // query range outside the q buffer: skip
-      return;
+      return false;
     }
     const int cap = min(L, max_query_len);
     if (Tq > cap) {
@@ -126,12 +156,12 @@ __global__ void __launch_bounds__(kThreads)
   }
   const int rows_total = Tq * group;
   const int row0 = qtile * 16;
-  if (row0 >= rows_total) return;
+  if (row0 >= rows_total) return false;
   const int nrows = min(16, rows_total - row0);  // rows of this tile (decode: = group)
 
   const int nblk_seq = (L + kBlockTokens - 1) / kBlockTokens;
   const int n_parts = nblk_seq > 0 ? (nblk_seq + part_blocks - 1) / part_blocks : 1;
-  if (part >= n_parts) return;
+  if (part >= n_parts) return false;
   const int blk_begin = part * part_blocks;
   const int nblk = min(nblk_seq - blk_begin, part_blocks);  // 0 only for an empty context
   const int q_head0 = kvh * group;
@@ -145,16 +175,18 @@ __global__ void __launch_bounds__(kThreads)
   const int n_mine = nblk > warp ? (nblk - warp + kWarps - 1) / kWarps : 0;
   uint8_t* wtiles = smem + warp * SM::kWarpBytes;
   uint64_t* wbars = bars + warp * SM::kStages;
-  if (lane == 0) {
+  if (init_bars) {
+    if (lane == 0) {
 #pragma unroll
-    for (int s = 0; s < SM::kStages; ++s) mbar_init(&wbars[s], 1);
-    fence_barrier_init();
-    if (warp == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      for (int s = 0; s < SM::kStages; ++s) mbar_init(&wbars[s], 1);
+      fence_barrier_init();
+      if (warp == 0) {
+        tma_prefetch_desc(tm_k);
+        tma_prefetch_desc(tm_v);
+      }
     }
+    __syncwarp();
   }
-  __syncwarp();
 
   // Physical block ids, 32 iterations per register window; ids outside the
   // pool are counted once (by the KV-head-0 CTA) and skipped.
@@ -178,15 +210,15 @@ __global__ void __launch_bounds__(kThreads)
     return __shfl_sync(kFull, v, it & 31);
   };
   auto issue = [&](int it, int p) {  // lane 0 only
-    const int st = it % SM::kStages;
+    const int st = (ring + it) % SM::kStages;
     uint8_t* kt = wtiles + st * SM::kStageBytes;
     uint8_t* vt = kt + SM::kTileBytes;
     if (p >= 0) {
       mbar_arrive_expect_tx(&wbars[st], 2 * SM::kTileBytes);
 #pragma unroll
       for (int c = 0; c < SM::kSubTiles; ++c) {
-        tma_load_4d(kt + c * 2048, &tm_k, &wbars[st], c * 64, 0, kvh, p);
-        tma_load_4d(vt + c * 2048, &tm_v, &wbars[st], c * 64, 0, kvh, p);
+        tma_load_4d(kt + c * 2048, tm_k, &wbars[st], c * 64, 0, kvh, p);
+        tma_load_4d(vt + c * 2048, tm_v, &wbars[st], c * 64, 0, kvh, p);
       }
     } else {
       mbar_arrive(&wbars[st]);  // nothing to load: complete the phase empty
@@ -234,8 +266,8 @@ __global__ void __launch_bounds__(kThreads)
       pid_cur = pid_nxt;
       pid_nxt = load_pid((win + 1) * 32 + lane);
     }
-    const int st = it % SM::kStages;
-    const uint32_t parity = (uint32_t)((it / SM::kStages) & 1);
+    const int st = (ring + it) % SM::kStages;
+    const uint32_t parity = (uint32_t)(((ring + it) / SM::kStages) & 1);
     const int p = pid_of(it);
     if (!__all_sync(kFull, mbar_wait(&wbars[st], parity))) {
       timed_out = true;
@@ -348,9 +380,11 @@ __global__ void __launch_bounds__(kThreads)
     // Let the copies already in flight land (each wait bounded) before the
     // shared memory is reused or the CTA exits, then report.
     const int last = min(n_mine, it + SM::kStages);
-    for (int k = it; k < last; ++k) (void)mbar_wait(&wbars[k % SM::kStages], (k / SM::kStages) & 1);
+    for (int k = it; k < last; ++k)
+      (void)mbar_wait(&wbars[(ring + k) % SM::kStages], ((ring + k) / SM::kStages) & 1);
     if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
   }
+  ring += (uint32_t)n_mine;
 
   // ---- merge the four warps (log-sum-exp), then write out or the partials
   l_a += __shfl_xor_sync(kFull, l_a, 1);
@@ -423,6 +457,186 @@ __global__ void __launch_bounds__(kThreads)
       *reinterpret_cast<float4*>(part_o + (orow * max_parts + part) * D + d) = res;
       if (d == 0) part_lse[orow * max_parts + part] = lsum > 0.f ? M + log2f(lsum) : -INFINITY;
     }
+  }
+  return timed_out;
+}
+
+// One CTA per work item: grid (max_parts * query tiles, KV heads, sequences).
+template <typename T, int D, bool kTwoRows, bool kMulti>
+__global__ void __launch_bounds__(kThreads)
+    decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, T* __restrict__ out,
+                            float* __restrict__ part_o, float* __restrict__ part_lse,
+                            const T* __restrict__ q, const int32_t* __restrict__ q_start,
+                            int num_q_tokens, int max_query_len,
+                            const int32_t* __restrict__ block_tables, int bt_stride,
+                            const int32_t* __restrict__ context_lens, int num_q_heads, int group,
+                            int64_t num_blocks, int max_context_len, float scale_log2,
+                            int part_blocks, int max_parts, int32_t* __restrict__ dev_error) {
+  using SM = DecodeSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOffset);
+  const ItemArgs<T> A{&tm_k,        &tm_v,     out,          part_o,        part_lse,
+                      q,            q_start,   num_q_tokens, max_query_len, block_tables,
+                      bt_stride,    context_lens, num_q_heads, group,       num_blocks,
+                      max_context_len, scale_log2, part_blocks, max_parts,  dev_error};
+  const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x;
+  const int qtile = kMulti ? (int)(blockIdx.x / (unsigned)max_parts) : 0;
+  uint32_t ring = 0;
+  (void)attend_item<T, D, kTwoRows, kMulti>(A, smem, bars, part, blockIdx.y, blockIdx.z, qtile,
+                                            true, ring);
+}
+
+// ---------------------------------------------------------------- work queue
+// Page-aware decode scheduling ("New Developments in 2026", PersistentKV:
+// pages, KV-head groups, sequence splits and work queues): a plan kernel
+// lists the (sequence, partition) items, longest first, and a persistent grid
+// of one wave of CTAs pulls (item, KV head) pairs from a global counter.
+// Empty partitions of short sequences cost nothing, and the long items start
+// first, so the last wave's tail is one short item.
+//
+// Plan layout (workspace): items[num_seqs * max_parts] = (seq << 16) | part,
+// then plan[0] = number of items, plan[1] = the work counter (zeroed here).
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 1024;  // item length in blocks, clamped; one bucket per thread
+
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void plan_counts(const int32_t* context_lens, int s,
+                                            int max_context_len, int part_blocks, int& n,
+                                            int& tail_blocks) {
+  int L = context_lens[s];
+  L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);  // as attend_item clamps
+  const int nblk = (L + kBlockTokens - 1) / kBlockTokens;
+  n = nblk > 0 ? (nblk + part_blocks - 1) / part_blocks : 1;
+  tail_blocks = nblk - (n - 1) * part_blocks;  // 0 for an empty context
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+    decode_plan_kernel(const int32_t* __restrict__ context_lens, int num_seqs,
+                       int max_context_len, int part_blocks, uint32_t* __restrict__ items,
+                       int32_t* __restrict__ plan) {
+  static_assert(kPlanThreads == kPlanBuckets, "one scan element per thread");
+  __shared__ int hist[kPlanBuckets];
+  __shared__ int cursor[kPlanBuckets];
+  __shared__ int warp_sum[kPlanThreads / 32];
+  griddep_launch_dependents();  // the decode grid may start its prologue now
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int full_bucket = min(part_blocks, kPlanBuckets - 1);
+  hist[tid] = 0;
+  __syncthreads();
+  for (int s = tid; s < num_seqs; s += kPlanThreads) {
+    int n, tail;
+    plan_counts(context_lens, s, max_context_len, part_blocks, n, tail);
+    if (n > 1) atomicAdd(&hist[full_bucket], n - 1);
+    atomicAdd(&hist[min(tail, kPlanBuckets - 1)], 1);
+  }
+  __syncthreads();
+  // cursor[b] = items in buckets above b (longer items first): an inclusive
+  // scan over the reversed bucket order, minus the bucket's own count.
+  const int b = kPlanBuckets - 1 - tid;
+  const int v = hist[b];
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sum[lane] = w;
+  }
+  __syncthreads();
+  const int incl = x + (warp > 0 ? warp_sum[warp - 1] : 0);
+  cursor[b] = incl - v;
+  if (tid == kPlanThreads - 1) {
+    plan[0] = incl;  // all items
+    plan[1] = 0;     // work counter
+  }
+  __syncthreads();
+  for (int s = tid; s < num_seqs; s += kPlanThreads) {
+    int n, tail;
+    plan_counts(context_lens, s, max_context_len, part_blocks, n, tail);
+    const uint32_t key = (uint32_t)s << 16;
+    if (n > 1) {
+      const int base = atomicAdd(&cursor[full_bucket], n - 1);
+      for (int p = 0; p < n - 1; ++p) items[base + p] = key | (uint32_t)p;
+    }
+    items[atomicAdd(&cursor[min(tail, kPlanBuckets - 1)], 1)] = key | (uint32_t)(n - 1);
+  }
+}
+
+// One wave of CTAs; each pulls work w -> (items[w / H_kv], KV head w % H_kv)
+// until the plan's items run out. A CTA's first work is its own index; each
+// later one comes from the counter, fetched one item ahead so the atomic's
+// latency hides behind the current item.
+template <typename T, int D, bool kTwoRows>
+__global__ void __launch_bounds__(kThreads)
+    decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, T* __restrict__ out,
+                             float* __restrict__ part_o, float* __restrict__ part_lse,
+                             const T* __restrict__ q, const int32_t* __restrict__ block_tables,
+                             int bt_stride, const int32_t* __restrict__ context_lens,
+                             int num_seqs, int num_q_heads, int group, int num_kv_heads,
+                             int64_t num_blocks, int max_context_len, float scale_log2,
+                             int part_blocks, int max_parts, const uint32_t* __restrict__ items,
+                             int32_t* __restrict__ plan, int32_t* __restrict__ dev_error) {
+  using SM = DecodeSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_next[2];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOffset);
+  const ItemArgs<T> A{&tm_k,        &tm_v,     out,      part_o,        part_lse,
+                      q,            nullptr,   num_seqs, 1,             block_tables,
+                      bt_stride,    context_lens, num_q_heads, group,   num_blocks,
+                      max_context_len, scale_log2, part_blocks, max_parts, dev_error};
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < SM::kStages; ++s) mbar_init(&bars[warp * SM::kStages + s], 1);
+    fence_barrier_init();
+    if (warp == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+  }
+  __syncwarp();
+  griddep_wait();  // the plan is complete and visible from here on
+
+  const int n_work = plan[0] * num_kv_heads;
+  int32_t* counter = plan + 1;
+  uint32_t ring = 0;
+  int w = blockIdx.x;
+  for (int k = 0; w < n_work; ++k) {
+    int nxt = 0;
+    if (threadIdx.x == 0) nxt = (int)gridDim.x + atomicAdd(counter, 1);
+    const uint32_t it = items[w / num_kv_heads];
+    const int seq = (int)(it >> 16), part = (int)(it & 0xffffu);
+    bool timed_out = false;
+    if (seq < num_seqs)
+      timed_out = attend_item<T, D, kTwoRows, false>(A, smem, bars, part, w % num_kv_heads, seq,
+                                                     0, false, ring);
+    // The item's generic shared-memory accesses (merge scratch, zeroed V
+    // rows) come before the next item's TMA writes to the same bytes.
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) s_next[k & 1] = nxt;
+    if (__syncthreads_or(timed_out)) break;
+    w = s_next[k & 1];
   }
 }
 
@@ -668,6 +882,68 @@ cudaError_t launch_reduce(const DecodeLaunch& a, cudaStream_t stream) {
                              : launch_reduce_typed<__nv_bfloat16, 64>(a, stream);
   return a.head_dim == 128 ? launch_reduce_typed<__half, 128>(a, stream)
                            : launch_reduce_typed<__half, 64>(a, stream);
+}
+
+template <typename T, int D, bool kTwoRows>
+static cudaError_t launch_persistent_typed(const DecodeLaunch& a, cudaStream_t stream) {
+  using SM = DecodeSmem<D>;
+  auto kern = decode_persistent_kernel<T, D, kTwoRows>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
+  if (e != cudaSuccess) return e;
+  static int per_sm = 0;  // resident CTAs per SM (the same on every device of this arch)
+  if (per_sm == 0) {
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, SM::kAlloc);
+    if (e != cudaSuccess) return e;
+    per_sm = n > 0 ? n : 1;
+  }
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const int64_t work_max = (int64_t)a.num_seqs * a.max_parts * a.num_kv_heads;
+  const int grid = (int)(work_max < (int64_t)sms * per_sm ? work_max : (int64_t)sms * per_sm);
+
+  decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(a.context_lens, a.num_seqs,
+                                                     a.max_context_len, a.part_blocks, a.items,
+                                                     a.plan);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // Programmatic dependent launch: the decode grid's prologue (barrier set-up,
+  // descriptor prefetch) overlaps the plan; griddepcontrol.wait orders the rest.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SM::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o,
+                         a.part_lse, static_cast<const T*>(a.q), a.block_tables, a.bt_stride,
+                         a.context_lens, a.num_seqs, a.num_q_heads, a.group, a.num_kv_heads,
+                         a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
+                         a.max_parts, static_cast<const uint32_t*>(a.items), a.plan,
+                         a.dev_error);
+  if (e != cudaSuccess) return e;
+  return launch_reduce_typed<T, D>(a, stream);
+}
+
+template <typename T>
+static cudaError_t launch_persistent_dtype(const DecodeLaunch& a, cudaStream_t stream) {
+  const bool two = a.group > 8;
+  if (a.head_dim == 128)
+    return two ? launch_persistent_typed<T, 128, true>(a, stream)
+               : launch_persistent_typed<T, 128, false>(a, stream);
+  return two ? launch_persistent_typed<T, 64, true>(a, stream)
+             : launch_persistent_typed<T, 64, false>(a, stream);
+}
+
+cudaError_t launch_decode_persistent(const DecodeLaunch& a, cudaStream_t stream) {
+  return a.bf16 ? launch_persistent_dtype<__nv_bfloat16>(a, stream)
+                : launch_persistent_dtype<__half>(a, stream);
 }
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {

@@ -38,9 +38,16 @@ struct DecodeLaunch {
   int32_t max_parts;
   int32_t* dev_error;
   int bf16;          // 0 = fp16, 1 = bf16
+  uint32_t* items;   // work queue: [num_seqs * max_parts] (seq << 16) | part
+  int32_t* plan;     // [0] = items listed, [1] = work counter
 };
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+
+// Decode (one query token per sequence) as a plan kernel that lists the
+// (sequence, partition) items longest first, a persistent grid that pulls
+// them from a counter, and the reduce. Uses a.items and a.plan.
+cudaError_t launch_decode_persistent(const DecodeLaunch& a, cudaStream_t stream);
 
 // The log-sum-exp reduce of split partitions alone (no-op for one partition).
 cudaError_t launch_reduce(const DecodeLaunch& a, cudaStream_t stream);

@@ -27,7 +27,8 @@ EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_bloc
            "pa_status_string", "pa_last_cuda_error", "pa_decode_static", "pa_swap_blocks",
            "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence",
            "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots", "pa_bm_append_slots",
-           "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount", "pa_prefill_chunk")
+           "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount", "pa_prefill_chunk",
+           "pa_decode_persistent_workspace_size", "pa_decode_persistent")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -61,6 +62,10 @@ def lib() -> ctypes.CDLL:
             L.pa_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, i32,
                                     ctypes.c_float, i32, P, sz, P, ctypes.c_int, P]
             L.pa_decode.restype = ctypes.c_int
+            L.pa_decode_persistent_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+            L.pa_decode_persistent_workspace_size.restype = sz
+            L.pa_decode_persistent.argtypes = L.pa_decode.argtypes
+            L.pa_decode_persistent.restype = ctypes.c_int
             L.pa_prefill_chunk.argtypes = [P, P, P, i32, i32, P, P, P, i32, P, i32, i32, i32,
                                            i32, i32, i64, i32, ctypes.c_float, i32, P, sz, P,
                                            ctypes.c_int, P]
@@ -156,9 +161,16 @@ def decode_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int, max_co
                                               partition_tokens))
 
 
+def decode_persistent_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int,
+                                     max_context_len: int, partition_tokens: int) -> int:
+    return int(lib().pa_decode_persistent_workspace_size(num_seqs, num_q_heads, head_dim,
+                                                         max_context_len, partition_tokens))
+
+
 def alloc_workspace(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens,
-                    device) -> torch.Tensor | None:
-    n = decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens)
+                    device, persistent: bool = False) -> torch.Tensor | None:
+    size = decode_persistent_workspace_size if persistent else decode_workspace_size
+    n = size(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens)
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
@@ -166,8 +178,11 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
            block_tables: torch.Tensor, context_lens: torch.Tensor, *, scale: float,
            max_context_len: int, partition_tokens: int = 512,
            workspace: torch.Tensor | None = None, dev_error: torch.Tensor | None = None,
-           stream=None) -> torch.Tensor:
-    """Paged decode attention: ``out [S, H_q, D] = attention(q, paged K/V)``."""
+           stream=None, persistent: bool = False) -> torch.Tensor:
+    """Paged decode attention: ``out [S, H_q, D] = attention(q, paged K/V)``.
+    ``persistent=True`` runs pa_decode_persistent (work-queue schedule, the
+    same result bit for bit); its workspace comes from
+    ``alloc_workspace(..., persistent=True)``."""
     S, Hq, D = q.shape
     NB, Hkv = k_cache.shape[:2]
     assert out.shape == q.shape and out.dtype == q.dtype == k_cache.dtype == v_cache.dtype
@@ -177,14 +192,15 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
     if Hq % Hkv:
         raise ValueError("num_q_heads must be a multiple of num_kv_heads")
     if workspace is None:
-        workspace = alloc_workspace(S, Hq, D, max_context_len, partition_tokens, q.device)
+        workspace = alloc_workspace(S, Hq, D, max_context_len, partition_tokens, q.device,
+                                    persistent)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-                         block_tables.shape[1], _ptr(context_lens), S, Hq, Hq // Hkv, D,
-                         PA_BLOCK_SIZE, NB, int(max_context_len), float(scale),
-                         int(partition_tokens), _ptr(workspace), ws_bytes, _ptr(dev_error),
-                         _dtype_code(q), _stream(stream, q.device))
-    _check(st, "pa_decode")
+    fn = lib().pa_decode_persistent if persistent else lib().pa_decode
+    st = fn(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            block_tables.shape[1], _ptr(context_lens), S, Hq, Hq // Hkv, D, PA_BLOCK_SIZE, NB,
+            int(max_context_len), float(scale), int(partition_tokens), _ptr(workspace), ws_bytes,
+            _ptr(dev_error), _dtype_code(q), _stream(stream, q.device))
+    _check(st, "pa_decode_persistent" if persistent else "pa_decode")
     return out
 
 

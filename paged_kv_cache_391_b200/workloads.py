@@ -393,6 +393,24 @@ def long_context(seed: int = 395, batch: int = 8, lo: int = 32768, hi: int = 131
                            dtype="bf16", seed=seed, pool_factor=pool_factor, rng=rng)
 
 
+def skewed(seed: int = 398, batch: int = 256, n_long: int = 4, long_lo: int = 65536,
+           long_hi: int = 131072, short_median: float = 512.0, sigma: float = 0.7,
+           short_hi: int = 4096) -> DecodeWorkload:
+    """A decode batch of mixed lengths on the Llama-3-8B GQA shape (32 query
+    heads over 8 KV heads, D = 128, bf16): ``n_long`` long-context requests
+    uniform in [65536, 131072] tokens among short ones, lognormal with median
+    512 (sigma 0.7) clipped to [16, 4096]; the long ones sit at random batch
+    positions. max_context_len is set by the longest, so a grid sized by it
+    holds mostly empty partitions: the case a work-queue schedule is for."""
+    rng = np.random.default_rng(seed)
+    lens = np.clip(np.round(np.exp(np.log(short_median) + sigma * rng.standard_normal(batch))),
+                   16, short_hi).astype(np.int64)
+    where = rng.choice(batch, size=n_long, replace=False)
+    lens[where] = rng.integers(long_lo, long_hi, size=n_long, endpoint=True)
+    return decode_workload("skewed", lens, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                           dtype="bf16", seed=seed, pool_factor=1.25, rng=rng)
+
+
 CONFIGS = {
     "tiny": tiny,
     "mha": mha,
@@ -401,6 +419,7 @@ CONFIGS = {
     "long": long_context,
     "spec_verify": spec_verify,
     "chunked_prefill": chunked_prefill,
+    "skewed": skewed,
 }
 
 

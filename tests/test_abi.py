@@ -134,3 +134,35 @@ def test_swap_blocks_rejects_on_the_host(L):
     assert f(*args(n=0)) == pa.PA_OK
     # an address no allocation owns is refused before any launch
     assert f(*args()) == pa.PA_ERR_INVALID_ARG
+
+
+def test_persistent_workspace_size(L):
+    f, base = L.pa_decode_persistent_workspace_size, L.pa_decode_workspace_size
+    assert f(0, 8, 128, 512, 512) == 0
+    # one partition: no partials, but the work list (8 items) and the plan
+    assert f(8, 64, 128, 512, 512) == 256 + 256
+    parts = 131072 // 512
+    assert f(8, 64, 128, 131072, 512) == (base(8, 64, 128, 131072, 512)
+                                           + -(-8 * parts * 4 // 256) * 256 + 256)
+
+
+def _decode_persistent(L, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, stride=4, cl=FAKE, S=2, Hq=8, g=4, D=128,
+             bs=16, NB=10, max_ctx=64, scale=0.1, P=512, ws=None, ws_bytes=0, err=None, dt=1)
+    a.update(kw)
+    return L.pa_decode_persistent(a["out"], a["q"], a["k"], a["v"], a["bt"], a["stride"],
+                                  a["cl"], a["S"], a["Hq"], a["g"], a["D"], a["bs"], a["NB"],
+                                  a["max_ctx"], ctypes.c_float(a["scale"]), a["P"], a["ws"],
+                                  a["ws_bytes"], a["err"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), pa.PA_ERR_INVALID_ARG),                                 # always needs a workspace
+    (dict(ws=FAKE + 16, ws_bytes=1 << 20), pa.PA_ERR_INVALID_ARG),   # not 256-byte aligned
+    (dict(ws=FAKE, ws_bytes=511), pa.PA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(max_ctx=16 * 65537, stride=65537, P=16), pa.PA_ERR_UNSUPPORTED),  # > 65536 partitions
+    (dict(g=3), pa.PA_ERR_UNSUPPORTED),
+    (dict(S=0), pa.PA_OK),
+])
+def test_decode_persistent_rejects_on_the_host(L, kw, status):
+    assert _decode_persistent(L, **kw) == status

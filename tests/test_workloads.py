@@ -145,3 +145,14 @@ def test_seeded_reproducible():
     a, b = W.tiny(), W.tiny()
     for f in ("k_pool", "v_pool", "q", "new_k", "block_tables", "slot_mapping"):
         assert np.array_equal(getattr(a, f), getattr(b, f))
+
+
+def test_skewed_structure():
+    w = W.skewed(batch=40, n_long=3, long_lo=2000, long_hi=3000, short_median=100,
+                 short_hi=500)
+    lens = w.context_lens
+    assert w.num_seqs == 40 and (w.num_q_heads, w.num_kv_heads, w.head_dim) == (32, 8, 128)
+    assert int((lens >= 2000).sum()) == 3 and lens.max() <= 3000
+    short = lens[lens < 2000]
+    assert short.min() >= 16 and short.max() <= 500
+    assert w.max_context_len == lens.max()
