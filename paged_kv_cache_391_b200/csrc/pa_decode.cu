@@ -663,17 +663,22 @@ __device__ __forceinline__ int seq_of_row(int row, int num_q_heads, const int32_
 }
 constexpr int kWarpRowMaxParts = 16;  // up to this many, one warp (half-warp) per row
 
+// Rows of up to kWarpRowMaxParts partitions: a warp (half-warp at D = 64)
+// per row, kReduceWarps rows per CTA; `cta` is this CTA's index among them.
 template <typename T, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32)
-    lse_reduce_kernel(T* __restrict__ out, const float* __restrict__ part_o,
-                      const float* __restrict__ part_lse, const int32_t* __restrict__ context_lens,
-                      const int32_t* __restrict__ q_start, int num_seqs, int num_rows,
-                      int num_q_heads, int max_context_len, int part_tokens, int max_parts) {
+__device__ __forceinline__ void reduce_rows_warp(T* __restrict__ out,
+                                                 const float* __restrict__ part_o,
+                                                 const float* __restrict__ part_lse,
+                                                 const int32_t* __restrict__ context_lens,
+                                                 const int32_t* __restrict__ q_start,
+                                                 int num_seqs, int num_rows, int num_q_heads,
+                                                 int max_context_len, int part_tokens,
+                                                 int max_parts, int cta) {
   constexpr int kLanes = D / 4;             // float4 columns of a row = lanes per row
   constexpr int kRowsPerWarp = 32 / kLanes;
   using E = Elem<T>;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row = (blockIdx.x * kReduceWarps + warp) * kRowsPerWarp + lane / kLanes;
+  const int row = (cta * kReduceWarps + warp) * kRowsPerWarp + lane / kLanes;
   const int c = lane % kLanes;
   const unsigned grp = kRowsPerWarp == 1 ? kFull : (0xffffu << (lane & ~(kLanes - 1)));
   int n = 0;
@@ -682,8 +687,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
     L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
     n = (L + part_tokens - 1) / part_tokens;
   }
-  // n is uniform within a row's lane group; rows with n <= 1 were written directly
-  if (n <= 1) return;
+  // n is uniform within a row's lane group; rows with n <= 1 were written
+  // directly, rows with more than kWarpRowMaxParts go to the split kernel
+  if (n <= 1 || n > kWarpRowMaxParts) return;
   const float* lse = part_lse + (size_t)row * max_parts;
   const float4* po = reinterpret_cast<const float4*>(part_o + (size_t)row * max_parts * D);
 
@@ -721,99 +727,135 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   *reinterpret_cast<uint2*>(out + (size_t)row * D + c * 4) = pk;
 }
 
-// Rows with many partitions (long contexts): one CTA per row. Phase 1 puts
-// the weights of all partitions in shared memory; phase 2 has every warp
-// (half-warp at D = 64) stream an interleaved subset of the partials; a
-// fixed-order merge of the streams ends it.
+// Rows with more than kWarpRowMaxParts partitions (long contexts): one CTA per
+// row at a time, `ncta` CTAs striding over the rows (rows with fewer
+// partitions are skipped). Phase 1 puts the weights of all partitions in
+// shared memory (s_w, max_parts floats); phase 2 has every warp (half-warp at
+// D = 64) stream an interleaved subset of the partials; a fixed-order merge
+// of the streams ends it.
 template <typename T, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32)
-    lse_reduce_split_kernel(T* __restrict__ out, const float* __restrict__ part_o,
-                            const float* __restrict__ part_lse,
-                            const int32_t* __restrict__ context_lens,
-                            const int32_t* __restrict__ q_start, int num_seqs, int num_q_heads,
-                            int max_context_len, int part_tokens, int max_parts) {
+__device__ __forceinline__ void reduce_rows_split(T* __restrict__ out,
+                                                  const float* __restrict__ part_o,
+                                                  const float* __restrict__ part_lse,
+                                                  const int32_t* __restrict__ context_lens,
+                                                  const int32_t* __restrict__ q_start,
+                                                  int num_seqs, int num_rows, int num_q_heads,
+                                                  int max_context_len, int part_tokens,
+                                                  int max_parts, int cta, int ncta, float* s_w) {
   constexpr int kThreadsR = kReduceWarps * 32;
   constexpr int kLanes = D / 4;
   constexpr int kStreams = kThreadsR / kLanes;
   using E = Elem<T>;
-  extern __shared__ float s_w[];  // [max_parts] weights
   __shared__ float s_red[kThreadsR];
   __shared__ float4 s_acc[kStreams][kLanes];
-  const int row = blockIdx.x;
-  int L = context_lens[seq_of_row(row, num_q_heads, q_start, num_seqs)];
-  L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
-  const int n = (L + part_tokens - 1) / part_tokens;
-  if (n <= 1) return;
   const int tid = threadIdx.x;
-  const float* lse = part_lse + (size_t)row * max_parts;
-  const float4* po = reinterpret_cast<const float4*>(part_o + (size_t)row * max_parts * D);
+  for (int row = cta; row < num_rows; row += ncta) {
+    int L = context_lens[seq_of_row(row, num_q_heads, q_start, num_seqs)];
+    L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
+    const int n = (L + part_tokens - 1) / part_tokens;
+    if (n <= kWarpRowMaxParts) continue;  // uniform over the CTA
+    const float* lse = part_lse + (size_t)row * max_parts;
+    const float4* po = reinterpret_cast<const float4*>(part_o + (size_t)row * max_parts * D);
 
-  // phase 1: M = max lse (fixed tree), weights, W = sum of weights (fixed tree)
-  float m = -INFINITY;
-  for (int p = tid; p < n; p += kThreadsR) {
-    const float l = lse[p];
-    s_w[p] = l;
-    m = fmaxf(m, l);
-  }
-  s_red[tid] = m;
-  __syncthreads();
-  for (int o = kThreadsR / 2; o > 0; o >>= 1) {
-    if (tid < o) s_red[tid] = fmaxf(s_red[tid], s_red[tid + o]);
+    // phase 1: M = max lse (fixed tree), weights, W = sum of weights (fixed tree)
+    float m = -INFINITY;
+    for (int p = tid; p < n; p += kThreadsR) {
+      const float l = lse[p];
+      s_w[p] = l;
+      m = fmaxf(m, l);
+    }
+    s_red[tid] = m;
     __syncthreads();
-  }
-  const float M = s_red[0];
-  __syncthreads();
-  float w = 0.f;
-  for (int p = tid; p < n; p += kThreadsR) {
-    const float l = s_w[p];
-    const float e = (M == -INFINITY || l == -INFINITY) ? 0.f : exp2f(l - M);
-    s_w[p] = e;
-    w += e;
-  }
-  s_red[tid] = w;
-  __syncthreads();
-  for (int o = kThreadsR / 2; o > 0; o >>= 1) {
-    if (tid < o) s_red[tid] += s_red[tid + o];
+    for (int o = kThreadsR / 2; o > 0; o >>= 1) {
+      if (tid < o) s_red[tid] = fmaxf(s_red[tid], s_red[tid + o]);
+      __syncthreads();
+    }
+    const float M = s_red[0];
     __syncthreads();
-  }
-  const float W = s_red[0];
+    float w = 0.f;
+    for (int p = tid; p < n; p += kThreadsR) {
+      const float l = s_w[p];
+      const float e = (M == -INFINITY || l == -INFINITY) ? 0.f : exp2f(l - M);
+      s_w[p] = e;
+      w += e;
+    }
+    s_red[tid] = w;
+    __syncthreads();
+    for (int o = kThreadsR / 2; o > 0; o >>= 1) {
+      if (tid < o) s_red[tid] += s_red[tid + o];
+      __syncthreads();
+    }
+    const float W = s_red[0];
 
-  // phase 2: independent weighted loads, one stream per warp (half-warp)
-  const int stream = tid / kLanes, c = tid % kLanes;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-  for (int p = stream; p < n; p += kStreams) {
-    const float wp = s_w[p];
-    const float4 v = po[(size_t)p * kLanes + c];
-    acc.x += wp * v.x;
-    acc.y += wp * v.y;
-    acc.z += wp * v.z;
-    acc.w += wp * v.w;
-  }
-  s_acc[stream][c] = acc;
-  __syncthreads();
-  if (tid < kLanes) {
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < kStreams; ++i) {
-      const float4 v = s_acc[i][tid];
-      a.x += v.x;
-      a.y += v.y;
-      a.z += v.z;
-      a.w += v.w;
+    // phase 2: independent weighted loads, one stream per warp (half-warp)
+    const int stream = tid / kLanes, c = tid % kLanes;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  #pragma unroll 8
+    for (int p = stream; p < n; p += kStreams) {
+      const float wp = s_w[p];
+      const float4 v = po[(size_t)p * kLanes + c];
+      acc.x += wp * v.x;
+      acc.y += wp * v.y;
+      acc.z += wp * v.z;
+      acc.w += wp * v.w;
     }
-    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (W > 0.f) {
-      res.x = a.x / W;
-      res.y = a.y / W;
-      res.z = a.z / W;
-      res.w = a.w / W;
+    s_acc[stream][c] = acc;
+    __syncthreads();
+    if (tid < kLanes) {
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  #pragma unroll
+      for (int i = 0; i < kStreams; ++i) {
+        const float4 v = s_acc[i][tid];
+        a.x += v.x;
+        a.y += v.y;
+        a.z += v.z;
+        a.w += v.w;
+      }
+      float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (W > 0.f) {
+        res.x = a.x / W;
+        res.y = a.y / W;
+        res.z = a.z / W;
+        res.w = a.w / W;
+      }
+      uint2 pk;
+      pk.x = E::pack(res.x, res.y);
+      pk.y = E::pack(res.z, res.w);
+      *reinterpret_cast<uint2*>(out + (size_t)row * D + tid * 4) = pk;
     }
-    uint2 pk;
-    pk.x = E::pack(res.x, res.y);
-    pk.y = E::pack(res.z, res.w);
-    *reinterpret_cast<uint2*>(out + (size_t)row * D + tid * 4) = pk;
+    __syncthreads();  // s_w, s_red and s_acc are reused by the next row
   }
+}
+
+// The reduce when no row can have more than kWarpRowMaxParts partitions.
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32)
+    lse_reduce_warp_kernel(T* __restrict__ out, const float* __restrict__ part_o,
+                           const float* __restrict__ part_lse,
+                           const int32_t* __restrict__ context_lens,
+                           const int32_t* __restrict__ q_start, int num_seqs, int num_rows,
+                           int num_q_heads, int max_context_len, int part_tokens, int max_parts) {
+  reduce_rows_warp<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
+                         num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x);
+}
+
+// The reduce otherwise, in one launch: CTAs [0, warp_ctas) take the rows of
+// up to kWarpRowMaxParts partitions, the others the rows of more.
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32)
+    lse_reduce_kernel(T* __restrict__ out, const float* __restrict__ part_o,
+                      const float* __restrict__ part_lse, const int32_t* __restrict__ context_lens,
+                      const int32_t* __restrict__ q_start, int num_seqs, int num_rows,
+                      int num_q_heads, int max_context_len, int part_tokens, int max_parts,
+                      int warp_ctas) {
+  extern __shared__ float s_w[];  // [max_parts] weights (split CTAs only)
+  if ((int)blockIdx.x < warp_ctas)
+    reduce_rows_warp<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
+                           num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x);
+  else
+    reduce_rows_split<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
+                            num_q_heads, max_context_len, part_tokens, max_parts,
+                            blockIdx.x - warp_ctas, gridDim.x - warp_ctas, s_w);
 }
 
 template <typename T, int D>
@@ -841,24 +883,33 @@ static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t strea
   cudaError_t e = cudaSuccess;
   if (a.max_parts <= 1) return e;
   const int rows = a.num_q_tokens * a.num_q_heads;
-  if (a.max_parts > kWarpRowMaxParts) {
-    const size_t wbytes = (size_t)a.max_parts * sizeof(float);
-    if (wbytes > 48 * 1024) {
-      e = cudaFuncSetAttribute(lse_reduce_split_kernel<T, D>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
-      if (e != cudaSuccess) return e;
-    }
-    lse_reduce_split_kernel<T, D><<<rows, kReduceWarps * 32, wbytes, stream>>>(
+  // Rows of up to kWarpRowMaxParts partitions: a warp (half-warp) each.
+  const int rows_per_cta = kReduceWarps * (32 / (D / 4));
+  const int warp_ctas = (rows + rows_per_cta - 1) / rows_per_cta;
+  if (a.max_parts <= kWarpRowMaxParts) {
+    lse_reduce_warp_kernel<T, D><<<warp_ctas, kReduceWarps * 32, 0, stream>>>(
         static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start, a.num_seqs,
-        a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts);
-  } else {
-    const int rows_per_cta = kReduceWarps * (32 / (D / 4));
-    lse_reduce_kernel<T, D><<<(rows + rows_per_cta - 1) / rows_per_cta, kReduceWarps * 32, 0,
-                              stream>>>(static_cast<T*>(a.out), a.part_o, a.part_lse,
-                                        a.context_lens, a.q_start, a.num_seqs, rows,
-                                        a.num_q_heads, a.max_context_len, a.part_tokens,
-                                        a.max_parts);
+        rows, a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts);
+    return cudaGetLastError();
   }
+  // Rows of more: a CTA each, one wave of CTAs striding over the rows.
+  auto kern = lse_reduce_kernel<T, D>;
+  const size_t wbytes = (size_t)a.max_parts * sizeof(float);
+  if (wbytes > 48 * 1024) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
+    if (e != cudaSuccess) return e;
+  }
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kReduceWarps * 32, wbytes);
+  if (e != cudaSuccess) return e;
+  const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+  const int split_ctas = (int)(rows < wave ? rows : wave);
+  kern<<<warp_ctas + split_ctas, kReduceWarps * 32, wbytes, stream>>>(
+      static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start, a.num_seqs, rows,
+      a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts, warp_ctas);
   return cudaGetLastError();
 }
 

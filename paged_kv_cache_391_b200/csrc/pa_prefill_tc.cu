@@ -8,18 +8,25 @@
 // With many query rows per KV head this is a dense contraction, so it runs on
 // tcgen05 instead of the 16-row mma.sync tiles of the decode kernel.
 //
-// One CTA per (128-row query tile, partition, KV head, sequence); tile rows are
-// (query token, head) pairs of the KV head's query group. 160 threads:
-//  * warps 0-3: softmax. Thread r owns row r: TMEM lane r of S, P and O.
-//  * warp 4, one lane: producer. It issues every TMA load (Q once; per step
-//    K and V of 4 cache blocks = 64 keys, each in its own 2-stage ring) and
-//    every MMA:
-//      S[j%2] = Q K_j^T   (M=128, N=64, K=D; Q and K K-major in shared memory)
-//      O     += P_j V_j   (M=128, N=D, K=64; P K-major, V MN-major)
+// One CTA per (pair of 128-row query tiles, partition, KV head, sequence);
+// tile rows are (query token, head) pairs of the KV head's query group. Both
+// tiles share every K/V tile the CTA loads, and while one tile's softmax runs
+// the tensor core works on the other's (the two-tile ping-pong of
+// FlashAttention-4). 320 threads, one CTA per SM:
+//  * warps 0-3 and 4-7: softmax of tile 0 and tile 1. Thread r of a
+//    warpgroup owns row r of its tile: TMEM lane r of its S, P and O.
+//  * warp 8: TMA loads (Q once; per step K and V of 4 cache blocks = 64 keys,
+//    each in its own 3-stage ring, eight lanes issuing a ring's eight boxes).
+//  * warp 9, one lane: every MMA, for tiles i = 0, 1:
+//      S_i[j%2] = Q_i K_j^T   (M=128, N=64, K=D; Q and K K-major in shared memory)
+//      O_i     += P_i,j V_j   (M=128, N=D, K=64; P K-major, V MN-major)
 //    S is double-buffered in TMEM so S(j+1) runs while the softmax of step j
-//    does; the softmax writes P_j (bf16, 128-byte swizzled) into one shared
-//    buffer once P.V(j-1) has read P_{j-1}. K_j's stage is refilled as soon as
-//    S(j) is done, V_j's once P.V(j) is, so S(j+2) never waits for P.V(j).
+//    does; each softmax writes P_i,j (bf16, 128-byte swizzled) into its
+//    tile's shared buffer once P.V(j-1) has read P_i,j-1. A K (V) stage is
+//    refilled once the S (P.V) MMAs that read it committed its "empty"
+//    barrier. Loads and MMAs sit in separate warps on separate schedulers,
+//    so neither waits on the other's instruction issue.
+//    TMEM: tile i at columns 256 i: S0 [0,64), S1 [64,128), O [128,256).
 // Online softmax per row in fp32, base 2 (hardware ex2); a row's reference
 // maximum and O are only rescaled when the maximum grows by more than 2^8.
 // Keys past the context, past the row's causal limit, or in a block with a bad
@@ -38,32 +45,39 @@
 namespace pa {
 namespace {
 
-constexpr int kRows = 128;                 // query rows per CTA (M)
+constexpr int kRows = 128;                 // query rows per tile (M)
+constexpr int kTiles = 2;                  // query tiles per CTA
 constexpr int kKeys = 64;                  // keys per step (4 cache blocks)
 constexpr int kStepBlocks = kKeys / 16;
 constexpr int kD = 128;                    // head dim of this path
 constexpr int kChunks = kD / 64;           // 128-byte swizzle columns of a row
-constexpr int kSoftmaxWarps = 4;
-constexpr int kThreadsTc = (kSoftmaxWarps + 1) * 32;
-constexpr uint32_t kTmemCols = 256;        // S0 [0,64) S1 [64,128) O [128,256)
+constexpr int kStages = 3;                 // K and V ring depth
+constexpr int kSoftmaxWarps = 4 * kTiles;
+constexpr int kLoadWarp = kSoftmaxWarps;       // TMA loads
+constexpr int kMmaWarp = kSoftmaxWarps + 1;    // tcgen05.mma issue
+constexpr int kThreadsTc = (kSoftmaxWarps + 2) * 32;
+constexpr uint32_t kTileCols = 256;        // per tile: S0 [0,64) S1 [64,128) O [128,256)
+constexpr uint32_t kTmemCols = kTiles * kTileCols;
 constexpr uint32_t kOCol = 128;
 
-constexpr int kQBytes = kRows * kD * 2;            // 32 KiB: [chunk][128 rows][128 B]
+constexpr int kQBytes = kRows * kD * 2;            // 32 KiB per tile: [chunk][128 rows][128 B]
 constexpr int kKBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]
 constexpr int kVBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]
-constexpr int kPBytes = kRows * kKeys * 2;        // 16 KiB: [128 rows][128 B] bf16 P
-constexpr int kQOff = 0;
-constexpr int kKOff = kQBytes;                     // K stages 0, 1
-constexpr int kVOff = kKOff + 2 * kKBytes;         // V stages 0, 1
-constexpr int kPOff = kVOff + 2 * kVBytes;
-constexpr int kBarOff = kPOff + kPBytes;
-// barriers: q_full, k_full[2], v_full[2], s_full[2], p_ready, pv_done; then the TMEM address
-constexpr int kNumBars = 9;
+constexpr int kPBytes = kRows * kKeys * 2;        // 16 KiB per tile: [128 rows][128 B] bf16 P
+constexpr int kQOff = 0;                           // Q tiles 0, 1
+constexpr int kKOff = kTiles * kQBytes;            // K stages
+constexpr int kVOff = kKOff + kStages * kKBytes;   // V stages
+constexpr int kPOff = kVOff + kStages * kVBytes;   // P tiles 0, 1
+constexpr int kBarOff = kPOff + kTiles * kPBytes;
+// barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3],
+// s_full[2 tiles][2], p_ready[2], pv_done[2]; then the TMEM address
+constexpr int kNumBars = 1 + 4 * kStages + 4 * kTiles;
 constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kTmemSlotOff + 16;
-// No alignment slack: two CTAs per SM need all of it. The dynamic shared
-// memory is declared 1024-byte aligned and the kernel checks it.
+// The dynamic shared memory is declared 1024-byte aligned and the kernel
+// checks it (no slack is reserved).
 constexpr int kSmemAlloc = kSmemBytes;
+static_assert(kSmemAlloc <= 227 * 1024, "one CTA per SM must fit");
 
 // 2^x by the hardware approximation (ex2.approx, relative error ~2^-22; 2^-inf = 0).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -79,7 +93,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 constexpr float kRescaleLog2 = 8.f;
 
 template <typename T>
-__global__ void __launch_bounds__(kThreadsTc)
+__global__ void __launch_bounds__(kThreadsTc, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, T* __restrict__ out,
@@ -94,11 +108,13 @@ __global__ void __launch_bounds__(kThreadsTc)
   uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* v_full = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;   // [2]
-  uint64_t* p_ready = bars + 7;
-  uint64_t* pv_done = bars + 8;
+  uint64_t* k_full = bars + 1;                      // [stage]
+  uint64_t* k_empty = k_full + kStages;             // [stage]
+  uint64_t* v_full = k_empty + kStages;             // [stage]
+  uint64_t* v_empty = v_full + kStages;             // [stage]
+  uint64_t* s_full = v_empty + kStages;             // [tile * 2 + buffer]
+  uint64_t* p_ready = s_full + 2 * kTiles;          // [tile]
+  uint64_t* pv_done = p_ready + kTiles;             // [tile]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlotOff);
 
   if (smem_addr(smem) & 1023) {  // the 128-byte swizzle needs 1024-byte aligned tiles
@@ -108,7 +124,7 @@ __global__ void __launch_bounds__(kThreadsTc)
   }
   const int kvh = blockIdx.y, seq = blockIdx.z;
   const int part = (int)(blockIdx.x % (unsigned)max_parts);
-  const int qtile = (int)(blockIdx.x / (unsigned)max_parts);
+  const int qtile = (int)(blockIdx.x / (unsigned)max_parts) * kTiles;  // the CTA's first tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool counter = part == 0 && kvh == 0 && qtile == 0 && tid == 0 && dev_error;
 
@@ -129,13 +145,13 @@ __global__ void __launch_bounds__(kThreadsTc)
     Tq = min(L, max_query_len);
   }
   const int tok_per_tile = kRows / group;
-  const int t0 = qtile * tok_per_tile;
+  const int t0 = qtile * tok_per_tile;  // first query token of the CTA
   if (t0 >= Tq) return;
   const int nblk_seq = (L + 15) / 16;
   const int n_parts = nblk_seq > 0 ? (nblk_seq + part_blocks - 1) / part_blocks : 1;
   if (part >= n_parts) return;
   const int key_begin = part * part_blocks * 16;
-  const int t_last = min(t0 + tok_per_tile, Tq) - 1;
+  const int t_last = min(t0 + kTiles * tok_per_tile, Tq) - 1;  // last query token of the CTA
   // keys this tile can see in this partition: up to the last row's causal limit
   const int key_end = min(min((part + 1) * part_blocks * 16, L), L - Tq + t_last + 1);
   const int n_steps = key_end > key_begin ? (key_end - key_begin + kKeys - 1) / kKeys : 0;
@@ -144,14 +160,18 @@ __global__ void __launch_bounds__(kThreadsTc)
   // ---- set-up: barriers (thread 0), TMEM (warp 0)
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(&k_full[0], 1);
-    mbar_init(&k_full[1], 1);
-    mbar_init(&v_full[0], 1);
-    mbar_init(&v_full[1], 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_ready, kSoftmaxWarps * 32);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < kTiles; ++i) {
+      mbar_init(&s_full[2 * i], 1);
+      mbar_init(&s_full[2 * i + 1], 1);
+      mbar_init(&p_ready[i], 4 * 32);
+      mbar_init(&pv_done[i], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -170,177 +190,186 @@ __global__ void __launch_bounds__(kThreadsTc)
   uint8_t* p_buf = smem + kPOff;
   const int32_t* bt_row = block_tables + (size_t)seq * bt_stride;
 
-  if (warp == kSoftmaxWarps) {
-    // =============================== producer ===============================
-    {
-      // The whole warp runs the producer's control flow (so the block table
-      // can be read 32 entries per coalesced load and broadcast by shuffle);
-      // lane 0 alone issues TMA loads, MMAs and commits.
-      const bool leader = lane == 0;
-      const uint32_t id_s = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kKeys, false, false);
-      const uint32_t id_pv = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kD, false, true);
-      // What is in flight, for the drain after a wait that gave up.
-      int k_pending[2] = {-1, -1}, v_pending[2] = {-1, -1};
-      uint64_t* last_bar = nullptr;  // barrier of the last MMA commit, and its parity
-      uint32_t last_parity = 0;
-      // Physical ids of the partition's blocks, 32 per register window: lane i
-      // holds entry 32 * win + i (-1 past the keys or for a bad entry).
-      const int lb_first = key_begin / 16;
-      const int nblk_keys = (key_end - key_begin + 15) / 16;
-      auto load_window = [&](int w) {
-        const int i = 32 * w + lane;
-        int p = -1;
-        if (i < nblk_keys) {
-          p = __ldg(bt_row + lb_first + i);
-          if (p < 0 || p >= num_blocks) p = -1;
-        }
-        return p;
-      };
-      int win = 0, pid_cur = load_window(0), pid_nxt = load_window(1);
-      auto pid_of = [&](int i) {  // all lanes; i within the current or the next window
-        const int v = (i >> 5) == win ? pid_cur : pid_nxt;
-        return __shfl_sync(0xffffffffu, v, i & 31);
-      };
-      // K (or V) of the step's four cache blocks into stage j % 2; blocks past
-      // the keys or with a bad table entry are not loaded.
-      auto load = [&](int j, bool is_v) {
-        const int st = j & 1;
-        uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
-        (is_v ? v_pending : k_pending)[st] = j;
-        uint8_t* dst = is_v ? stage_v(st) : stage_k(st);
-        const CUtensorMap* map = is_v ? &tm_v : &tm_k;
-        while (((j * kStepBlocks) >> 5) > win) {  // a step's 4 entries share one window
-          ++win;                       // slide the table window forward
-          pid_cur = pid_nxt;
-          pid_nxt = load_window(win + 1);
-        }
-        int pids[kStepBlocks];
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int b = 0; b < kStepBlocks; ++b) {
-          pids[b] = pid_of(j * kStepBlocks + b);
-          if (pids[b] >= 0) bytes += kChunks * 2048;
-        }
-        if (!leader) return;
-        if (bytes == 0) {
-          mbar_arrive(bar);
-          return;
-        }
-        mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-        for (int b = 0; b < kStepBlocks; ++b) {
-          if (pids[b] < 0) continue;
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_4d(dst + c * (kKeys * 128) + b * 2048, map, bar, c * 64, 0, kvh, pids[b]);
-        }
-      };
-      // Every wait is taken by all lanes and agreed on, so the warp stays converged.
-      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity));
-      };
-      auto wait_k = [&](int j) {
-        const bool ok = wait_all(&k_full[j & 1], (j >> 1) & 1);
-        if (ok) k_pending[j & 1] = -1;
-        return ok;
-      };
-      auto wait_v = [&](int j) {
-        const bool ok = wait_all(&v_full[j & 1], (j >> 1) & 1);
-        if (ok) v_pending[j & 1] = -1;
-        return ok;
-      };
-      auto issue_s = [&](int j) {
-        const int st = j & 1;
-        last_bar = &s_full[st];
-        last_parity = (uint32_t)((j >> 1) & 1);
-        if (!leader) return;
-        const uint32_t k_s = smem_addr(stage_k(st));
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;  // 16 columns = 32 bytes into the swizzled row
-          const uint64_t a = tc::smem_desc_sw128(q_s + (kk >> 2) * (kRows * 128) + off, 16, 1024);
-          const uint64_t b = tc::smem_desc_sw128(k_s + (kk >> 2) * (kKeys * 128) + off, 16, 1024);
-          tc::mma_f16(tmem + (uint32_t)(st * kKeys), a, b, id_s, kk > 0);
-        }
-        tc::commit(&s_full[st]);
-      };
-      auto issue_pv = [&](int j) {
-        const int st = j & 1;
-        last_bar = pv_done;
-        last_parity = (uint32_t)(j & 1);
-        if (!leader) return;
-        const uint32_t v_s = smem_addr(stage_v(st));
-        const uint32_t p_s = smem_addr(p_buf);
-#pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t a = tc::smem_desc_sw128(p_s + kk * 32, 16, 1024);
-          const uint64_t b = tc::smem_desc_sw128(v_s + kk * 2048, kKeys * 128, 1024);
-          tc::mma_f16(tmem + kOCol, a, b, id_pv, j > 0 || kk > 0);
-        }
-        tc::commit(pv_done);
-      };
-
-      if (leader) tma_prefetch_desc(&tm_q);
-      if (n_steps > 0) {
-        if (leader) {
-          mbar_arrive_expect_tx(q_full, kQBytes);
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c)
-            tc::tma_load_3d(smem + kQOff + c * (kRows * 128), &tm_q, q_full, c * 64, q_head0,
-                            q0 + t0);
-        }
-        load(0, false);
-        load(0, true);
-        if (n_steps > 1) {
-          load(1, false);
-          load(1, true);
-        }
-        failed = !wait_all(q_full, 0) || !wait_k(0);
-        if (!failed) issue_s(0);
+  if (warp == kLoadWarp) {
+    // ============================ TMA loads =================================
+    // The whole warp runs the control flow, so the block table is read 32
+    // entries per coalesced load and broadcast by shuffle. Per step and ring
+    // (K, then V) lane 0 posts the expected bytes and lanes 0-7 issue the
+    // step's eight box copies (4 cache blocks x 2 column chunks) in one
+    // instruction. A stage is refilled once the MMAs that read it committed
+    // its "empty" barrier; the loads run up to kStages steps ahead.
+    const int lb_first = key_begin / 16;
+    const int nblk_keys = (key_end - key_begin + 15) / 16;
+    auto load_window = [&](int w) {
+      const int i = 32 * w + lane;
+      int p = -1;
+      if (i < nblk_keys) {
+        p = __ldg(bt_row + lb_first + i);
+        if (p < 0 || p >= num_blocks) p = -1;
       }
-      for (int j = 0; j < n_steps && !failed; ++j) {
-        // S(j+1): its TMEM buffer was read by softmax(j-1), whose p_ready was
-        // awaited in the previous iteration.
-        if (j + 1 < n_steps) {
-          if (!wait_k(j + 1)) { failed = true; break; }
-          issue_s(j + 1);
-        }
-        // V(j+1) into the stage PV(j-1) has finished reading
-        if (j >= 1 && j + 1 < n_steps) {
-          if (!wait_all(pv_done, (j - 1) & 1)) { failed = true; break; }
-          load(j + 1, true);
-        }
-        // K(j+2) into the stage S(j) has finished reading
-        if (j + 2 < n_steps) {
-          if (!wait_all(&s_full[j & 1], (j >> 1) & 1)) { failed = true; break; }
-          load(j + 2, false);
-        }
-        if (!wait_all(p_ready, j & 1) || !wait_v(j)) { failed = true; break; }
+      return p;
+    };
+    int win = 0, pid_cur = load_window(0), pid_nxt = load_window(1);
+    auto pid_of = [&](int i) {  // all lanes; i / 32 uniform over the warp
+      const int w = i >> 5;
+      if (w != win && w != win + 1) {  // outside the register window: read the table
+        const int p = i < nblk_keys ? __ldg(bt_row + lb_first + i) : -1;
+        return (p < 0 || p >= num_blocks) ? -1 : p;
+      }
+      const int v = w == win ? pid_cur : pid_nxt;
+      return __shfl_sync(0xffffffffu, v, i & 31);
+    };
+    // K (or V) of step j's four cache blocks into stage j % kStages; blocks
+    // past the keys or with a bad table entry are not loaded.
+    auto load = [&](int j, bool is_v) {
+      const int st = j % kStages;
+      uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
+      uint8_t* dst = is_v ? stage_v(st) : stage_k(st);
+      const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+      while (((j * kStepBlocks) >> 5) > win) {  // a step's 4 entries share one window
+        ++win;
+        pid_cur = pid_nxt;
+        pid_nxt = load_window(win + 1);
+      }
+      const int b = (lane >> 1) & (kStepBlocks - 1), c = lane & 1;  // lanes 0-7: block, chunk
+      const int pid = pid_of(j * kStepBlocks + b);
+      const bool mine = lane < kStepBlocks * kChunks && pid >= 0;
+      const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, mine)) * 2048u;
+      if (lane == 0) {
+        if (bytes) mbar_arrive_expect_tx(bar, bytes);
+        else mbar_arrive(bar);  // nothing to load: complete the phase empty
+      }
+      __syncwarp();
+      if (mine) tma_load_4d(dst + c * (kKeys * 128) + b * 2048, map, bar, c * 64, 0, kvh, pid);
+    };
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    int nk = 0, nv = 0;  // steps whose K / V loads were issued
+    if (n_steps > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        // Both tiles' rows; rows past the q buffer read as zeros (and are
+        // never written out).
+        mbar_arrive_expect_tx(q_full, kTiles * kQBytes);
+#pragma unroll
+        for (int i = 0; i < kTiles; ++i)
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c)
+            tc::tma_load_3d(smem + kQOff + i * kQBytes + c * (kRows * 128), &tm_q, q_full,
+                            c * 64, q_head0, q0 + t0 + i * tok_per_tile);
+      }
+      for (int j = 0; j < n_steps; ++j) {
+        const uint32_t reuse = (uint32_t)((j / kStages - 1) & 1);
+        if (j >= kStages && !wait_all(&k_empty[j % kStages], reuse)) { failed = true; break; }
+        load(j, false);
+        ++nk;
+        if (j >= kStages && !wait_all(&v_empty[j % kStages], reuse)) { failed = true; break; }
+        load(j, true);
+        ++nv;
+      }
+    }
+    if (failed) {
+      // Let the copies already issued land (each wait bounded) before the
+      // shared memory is released.
+      (void)mbar_wait(q_full, 0);
+      for (int st = 0; st < kStages; ++st) {
+        // the last load issued into stage st is step st + kStages * ((n - 1 - st) / kStages)
+        if (nk > st) (void)mbar_wait(&k_full[st], (uint32_t)(((nk - 1 - st) / kStages) & 1));
+        if (nv > st) (void)mbar_wait(&v_full[st], (uint32_t)(((nv - 1 - st) / kStages) & 1));
+      }
+      if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
+    }
+  } else if (warp == kMmaWarp) {
+    // ============================== MMAs ====================================
+    // One lane issues every tcgen05.mma, in the order S(j) of both tiles,
+    // then P.V(j-1) of both tiles, so S(j) runs while the softmax of step
+    // j-1 finishes. Descriptors are built once and offset per MMA.
+    const bool leader = lane == 0;
+    const uint32_t id_s = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kKeys, false, false);
+    const uint32_t id_pv = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kD, false, true);
+    const uint64_t dq = tc::smem_desc_sw128(q_s, 16, 1024);
+    const uint64_t dk = tc::smem_desc_sw128(smem_addr(stage_k(0)), 16, 1024);
+    const uint64_t dv = tc::smem_desc_sw128(smem_addr(stage_v(0)), kKeys * 128, 1024);
+    const uint64_t dp = tc::smem_desc_sw128(smem_addr(p_buf), 16, 1024);
+    uint64_t* last_bar = nullptr;  // barrier of the last commit, and its parity
+    uint32_t last_parity = 0;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    if (n_steps > 0 && !wait_all(q_full, 0)) failed = true;
+    for (int j = 0; j <= n_steps && !failed; ++j) {
+      if (j < n_steps) {
+        // S(j): its TMEM buffer j % 2 was read by softmax(j-2), whose p_ready
+        // was awaited before P.V(j-2).
+        const int st = j % kStages, buf = j & 1;
+        if (!wait_all(&k_full[st], (uint32_t)((j / kStages) & 1))) { failed = true; break; }
         tc::fence_after_sync();
-        issue_pv(j);
-      }
-      if (failed) {
-        // Let the copies and MMAs already issued finish (each wait bounded)
-        // before shared memory and TMEM are released.
-        (void)mbar_wait(q_full, 0);
-        for (int st = 0; st < 2; ++st) {
-          if (k_pending[st] >= 0) (void)mbar_wait(&k_full[st], (k_pending[st] >> 1) & 1);
-          if (v_pending[st] >= 0) (void)mbar_wait(&v_full[st], (v_pending[st] >> 1) & 1);
+        if (leader) {
+          const uint64_t dks = dk + (uint64_t)((st * kKBytes) >> 4);
+#pragma unroll
+          for (int i = 0; i < kTiles; ++i) {
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = (kk & 3) * 32;  // 16 columns = 32 bytes into the row
+              const uint64_t a = dq + (uint64_t)((i * kQBytes + (kk >> 2) * (kRows * 128) + off) >> 4);
+              const uint64_t b = dks + (uint64_t)(((kk >> 2) * (kKeys * 128) + off) >> 4);
+              tc::mma_f16(tmem + (uint32_t)(i * kTileCols + buf * kKeys), a, b, id_s, kk > 0);
+            }
+            tc::commit(&s_full[2 * i + buf]);
+          }
+          tc::commit(&k_empty[st]);  // K stage st free once these MMAs completed
         }
-        if (last_bar) (void)mbar_wait(last_bar, last_parity);
-        if (leader && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
+        last_bar = &k_empty[st];
+        last_parity = (uint32_t)((j / kStages) & 1);
       }
+      if (j >= 1) {
+        // P.V(j-1) of both tiles, once V(j-1) landed and each tile's P is in place
+        const int jp = j - 1, st = jp % kStages;
+        if (!wait_all(&v_full[st], (uint32_t)((jp / kStages) & 1))) { failed = true; break; }
+        const uint64_t dvs = dv + (uint64_t)((st * kVBytes) >> 4);
+        for (int i = 0; i < kTiles; ++i) {
+          if (!wait_all(&p_ready[i], (uint32_t)(jp & 1))) { failed = true; break; }
+          tc::fence_after_sync();
+          if (leader) {
+#pragma unroll
+            for (int kk = 0; kk < kKeys / 16; ++kk) {
+              const uint64_t a = dp + (uint64_t)((i * kPBytes + kk * 32) >> 4);
+              const uint64_t b = dvs + (uint64_t)((kk * 2048) >> 4);
+              tc::mma_f16(tmem + (uint32_t)(i * kTileCols) + kOCol, a, b, id_pv, jp > 0 || kk > 0);
+            }
+            tc::commit(&pv_done[i]);
+          }
+          last_bar = &pv_done[i];
+          last_parity = (uint32_t)(jp & 1);
+        }
+        if (failed) break;
+        if (leader) tc::commit(&v_empty[st]);
+        last_bar = &v_empty[st];
+        last_parity = (uint32_t)((jp / kStages) & 1);
+      }
+    }
+    if (failed) {
+      // The MMAs already issued finish (bounded wait) before TMEM is released.
+      if (last_bar) (void)mbar_wait(last_bar, last_parity);
+      if (leader && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
     }
   } else {
     // =============================== softmax ================================
-    const int r = tid;                                   // tile row = TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    const int t = t0 + r / group, h = r % group;         // query token in the chunk, head
+    const int tile = warp >> 2;                          // this warpgroup's query tile
+    const int r = tid & (kRows - 1);                     // tile row = TMEM lane
+    const uint32_t lane_addr =
+        tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(tile * kTileCols);
+    const int tt0 = t0 + tile * tok_per_tile;            // first query token of the tile
+    const int t = tt0 + r / group, h = r % group;        // query token in the chunk, head
     const bool row_ok = t < Tq;
     const int lim = L - Tq + (row_ok ? t : 0);           // last key this row may see
     float m = -INFINITY, l = 0.f;                        // reference maximum (log2 units)
     // keys every row of the tile may see: up to the first row's causal limit
-    const int key_all = min(key_end, L - Tq + t0 + 1);
+    const int key_all = min(key_end, L - Tq + tt0 + 1);
+    uint64_t* my_s_full = &s_full[2 * tile];
+    uint64_t* my_pv_done = &pv_done[tile];
+    uint8_t* my_p = p_buf + tile * kPBytes;
     // Validity of the table entries of a step (a bit per cache block), loaded
     // one step ahead so the table reads never wait in the loop.
     auto bad_blocks = [&](int j) {
@@ -358,17 +387,17 @@ __global__ void __launch_bounds__(kThreadsTc)
     };
     int bad_next = n_steps > 0 ? bad_blocks(0) : 0;
     for (int j = 0; j < n_steps; ++j) {
-      const int st = j & 1;
+      const int buf = j & 1, st = j % kStages;
       const int kb = key_begin + j * kKeys;
       const int bad_mask = bad_next;
       if (j + 1 < n_steps) bad_next = bad_blocks(j + 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1))) { failed = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&my_s_full[buf], (j >> 1) & 1))) { failed = true; break; }
       tc::fence_after_sync();
       float s[64];
       {
         float a[32], b2[32];
-        tc::tmem_ld32(lane_addr + (uint32_t)(st * kKeys), a);
-        tc::tmem_ld32(lane_addr + (uint32_t)(st * kKeys + 32), b2);
+        tc::tmem_ld32(lane_addr + (uint32_t)(buf * kKeys), a);
+        tc::tmem_ld32(lane_addr + (uint32_t)(buf * kKeys + 32), b2);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -419,12 +448,12 @@ __global__ void __launch_bounds__(kThreadsTc)
       }
       l = l * alpha + psum;
       // PV(j-1) must be done before O is rescaled (it writes O).
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) { failed = true; break; }
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(my_pv_done, (j - 1) & 1))) { failed = true; break; }
       tc::fence_after_sync();
       // P_j row r: 64 bf16 = 128 bytes, 128-byte swizzle (PV(j-1) has read P_{j-1})
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(p_buf + r * 128 + ((c ^ (r & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(my_p + r * 128 + ((c ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       // rescale O when a row's reference maximum moved (warp-uniform decision)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -439,11 +468,13 @@ __global__ void __launch_bounds__(kThreadsTc)
         }
       }
       if (j > 0) tc::tmem_wait_st();
-      // V rows of keys past the context or of bad blocks become zero (once V_j landed)
-      if (kb + kKeys > key_end || bad_mask) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (j >> 1) & 1))) { failed = true; break; }
+      // V rows of keys past the context or of bad blocks become zero (once V_j
+      // landed); tile 0 does it, before its p_ready, which the MMA warp awaits
+      // before either tile's P.V(j).
+      if (tile == 0 && (kb + kKeys > key_end || bad_mask)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (j / kStages) & 1))) { failed = true; break; }
         uint8_t* v = stage_v(st);
-        for (int i = r; i < kKeys * kChunks * 8; i += kSoftmaxWarps * 32) {
+        for (int i = r; i < kKeys * kChunks * 8; i += kRows) {
           const int c = i / (kKeys * 8), rem = i % (kKeys * 8);
           const int key = rem / 8;
           if (kb + key >= key_end || ((bad_mask >> (key >> 4)) & 1))
@@ -453,11 +484,11 @@ __global__ void __launch_bounds__(kThreadsTc)
       }
       fence_proxy_async_smem();  // P (and zeroed V rows) -> visible to the tensor core
       tc::fence_before_sync();
-      mbar_arrive(p_ready);
+      mbar_arrive(&p_ready[tile]);
     }
     // ---- epilogue: O / l  ->  out (one partition) or fp32 partials
     if (!failed && n_steps > 0 &&
-        !__all_sync(0xffffffffu, mbar_wait(pv_done, (n_steps - 1) & 1)))
+        !__all_sync(0xffffffffu, mbar_wait(my_pv_done, (n_steps - 1) & 1)))
       failed = true;
     if (failed) {
       if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
@@ -525,7 +556,8 @@ cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q,
                                          kSmemAlloc);
     if (e != cudaSuccess) return e;
     const int qtiles = (a.max_query_len * a.group + kRows - 1) / kRows;
-    dim3 grid((unsigned)((int64_t)a.max_parts * qtiles), a.num_kv_heads, a.num_seqs);
+    const int pairs = (qtiles + kTiles - 1) / kTiles;
+    dim3 grid((unsigned)((int64_t)a.max_parts * pairs), a.num_kv_heads, a.num_seqs);
     kern<<<grid, kThreadsTc, kSmemAlloc, stream>>>(
         tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, a.q_start,
         a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride, a.context_lens,

@@ -94,3 +94,13 @@ def test_tensor_core_chunks_scale_zero_and_large_logits(scale):
                          head_dim=128, dtype="bf16", seed=int(scale) + 40)
     w.scale = scale
     _check(w)
+
+
+@pytest.mark.parametrize("P", [0, 512])
+def test_tensor_core_tile_pairs(P):
+    """The tcgen05 kernel takes query tiles two at a time: 3, 5 and 9 tiles of
+    128 (token, head) rows leave the last pair's second tile empty or partly
+    filled, and its rows past the chunk (or in the next sequence) unwritten."""
+    w = W.chunk_workload("pairs", [300, 1000, 2500], [96, 160, 288], num_q_heads=8,
+                         num_kv_heads=2, head_dim=128, dtype="bf16", seed=50 + P)
+    _check(w, P)
