@@ -290,15 +290,28 @@ __device__ __forceinline__ bool attend_item(const ItemArgs<T>& A, uint8_t* smem,
         __syncwarp();
       }
 
-      // S = Q K^T for the 16 tokens: two n-tiles of 8 tokens, K over D.
+      // S = Q K^T for the 16 tokens: two n-tiles of 8 tokens, K over D; the
+      // even and odd K steps accumulate separately (two dependency chains of
+      // D/32 tensor-core ops instead of one of D/16), then add.
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      float u0[4] = {0.f, 0.f, 0.f, 0.f}, u1[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t kbase = smem_addr(kt);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4(kbase + tile_off((mi >> 1) * 8 + r8, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
-        E::mma(s0, qa[kk], b0, b1);
-        E::mma(s1, qa[kk], b2, b3);
+        if (kk & 1) {
+          E::mma(u0, qa[kk], b0, b1);
+          E::mma(u1, qa[kk], b2, b3);
+        } else {
+          E::mma(s0, qa[kk], b0, b1);
+          E::mma(s1, qa[kk], b2, b3);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        s0[i] += u0[i];
+        s1[i] += u1[i];
       }
 
       // Online softmax (base 2). Lane holds, for head row a = gid (and
