@@ -89,7 +89,9 @@ def make_workload(name, batch, seed_offset=0):
 
 
 KERNEL_SOURCES = ("paged_kv_cache_391_b200/csrc/pa_decode.cu",
-                  "paged_kv_cache_391_b200/csrc/pa_device.cuh")
+                  "paged_kv_cache_391_b200/csrc/pa_device.cuh",
+                  "paged_kv_cache_391_b200/csrc/pa_prefill_tc.cu",
+                  "paged_kv_cache_391_b200/csrc/pa_tcgen05.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
@@ -662,9 +664,10 @@ def main():
             "flops_per_launch": flops,
             "algorithmic_bytes_per_launch": sb["decode"],
             "traffic": recorded_traffic(args.workload, args.batch, args.scheduler),
-            "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                            "decode_partition_kernel + lse_reduce per call "
-                            "(profiles/dram_traffic.txt; null if the kernel changed since)",
+            "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
+                            "call's kernels (partition or persistent kernel, plan, LSE "
+                            "reduce) per call, full-size workload (profiles/dram_traffic.txt; "
+                            "null if a kernel source changed since)",
         },
         "sub_ms": {"decode": round(dec_ms, 5),
                    "write_kv_and_copies": round(elapsed_ms / K - dec_ms, 5)},
