@@ -88,29 +88,35 @@ def make_workload(name, batch, seed_offset=0):
     return fn(seed=seed, **kw)
 
 
-KERNEL_SOURCES = ("paged_kv_cache_391_b200/csrc/pa_decode.cu",
-                  "paged_kv_cache_391_b200/csrc/pa_device.cuh",
-                  "paged_kv_cache_391_b200/csrc/pa_prefill_tc.cu",
-                  "paged_kv_cache_391_b200/csrc/pa_tcgen05.cuh")
+# The sources each kernel family is built from: a recorded traffic figure is
+# valid only while the hash of its family's sources is unchanged.
+KERNEL_SOURCES = {
+    "mma": ("paged_kv_cache_391_b200/csrc/pa_decode.cu",
+            "paged_kv_cache_391_b200/csrc/pa_device.cuh"),
+    "tcgen05": ("paged_kv_cache_391_b200/csrc/pa_prefill_tc.cu",
+                "paged_kv_cache_391_b200/csrc/pa_tcgen05.cuh",
+                "paged_kv_cache_391_b200/csrc/pa_device.cuh"),
+}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+TC_WORKLOADS = ("chunked_prefill",)  # the configs whose chunks take the tcgen05 kernel
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(family: str = "mma") -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[family]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str, batch, scheduler: str = "grid"):
-    """DRAM bytes (read + write) per pa_decode call from the ncu capture
+    """DRAM bytes (read + write) per attention call from the ncu capture
     recorded in profiles/dram_traffic.txt for this workload, or None when
-    there is none or the kernel sources changed since it was taken."""
+    there is none or its kernel sources changed since it was taken."""
     if batch is not None or not os.path.exists(TRAFFIC_FILE):
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash("tcgen05" if workload in TC_WORKLOADS else "mma")
     key = workload if scheduler == "grid" else f"{workload}:{scheduler}"
     with open(TRAFFIC_FILE) as f:
         for line in f:

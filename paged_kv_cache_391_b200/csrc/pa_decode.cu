@@ -852,23 +852,25 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
                          num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x);
 }
 
-// The reduce otherwise, in one launch: CTAs [0, warp_ctas) take the rows of
-// up to kWarpRowMaxParts partitions, the others the rows of more.
+// The reduce otherwise, in one launch: CTAs [0, split_ctas) stride over the
+// rows of more than kWarpRowMaxParts partitions (dispatched first: those rows
+// are the long pole), the others take the rows of up to kWarpRowMaxParts.
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
     lse_reduce_kernel(T* __restrict__ out, const float* __restrict__ part_o,
                       const float* __restrict__ part_lse, const int32_t* __restrict__ context_lens,
                       const int32_t* __restrict__ q_start, int num_seqs, int num_rows,
                       int num_q_heads, int max_context_len, int part_tokens, int max_parts,
-                      int warp_ctas) {
+                      int split_ctas) {
   extern __shared__ float s_w[];  // [max_parts] weights (split CTAs only)
-  if ((int)blockIdx.x < warp_ctas)
-    reduce_rows_warp<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
-                           num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x);
-  else
+  if ((int)blockIdx.x < split_ctas)
     reduce_rows_split<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
-                            num_q_heads, max_context_len, part_tokens, max_parts,
-                            blockIdx.x - warp_ctas, gridDim.x - warp_ctas, s_w);
+                            num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x,
+                            split_ctas, s_w);
+  else
+    reduce_rows_warp<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
+                           num_q_heads, max_context_len, part_tokens, max_parts,
+                           blockIdx.x - split_ctas);
 }
 
 template <typename T, int D>
@@ -922,7 +924,7 @@ static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t strea
   const int split_ctas = (int)(rows < wave ? rows : wave);
   kern<<<warp_ctas + split_ctas, kReduceWarps * 32, wbytes, stream>>>(
       static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start, a.num_seqs, rows,
-      a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts, warp_ctas);
+      a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts, split_ctas);
   return cudaGetLastError();
 }
 
