@@ -29,6 +29,8 @@
 //    depend on which physical blocks hold the context, bit for bit.
 #include <math.h>
 
+#include <utility>
+
 #include "pa.h"
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -72,6 +74,17 @@ struct DecodeSmem {
 // within a row is XORed with (row % 8), as TMA's 128-byte swizzle lays it out.
 __device__ __forceinline__ uint32_t tile_off(int t, int d) {
   return (uint32_t)((d >> 6) * 2048 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4) + (d & 7) * 2);
+}
+
+// Programmatic dependent launch: a kernel launched with the attribute may
+// start while the previous kernel in the stream finishes; it reads no global
+// memory before griddep_wait(), which returns once that kernel has completed
+// and its writes are visible. Without the attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // The arguments every work item shares.
@@ -497,9 +510,23 @@ __global__ void __launch_bounds__(kThreads)
                       max_context_len, scale_log2, part_blocks, max_parts,  dev_error};
   const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x;
   const int qtile = kMulti ? (int)(blockIdx.x / (unsigned)max_parts) : 0;
+  // Barriers and descriptor prefetch before the dependency wait: they touch
+  // no memory the previous kernel writes.
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < SM::kStages; ++s) mbar_init(&bars[warp * SM::kStages + s], 1);
+    fence_barrier_init();
+    if (warp == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+  }
+  __syncwarp();
+  griddep_wait();
   uint32_t ring = 0;
   (void)attend_item<T, D, kTwoRows, kMulti>(A, smem, bars, part, blockIdx.y, blockIdx.z, qtile,
-                                            true, ring);
+                                            false, ring);
 }
 
 // ---------------------------------------------------------------- work queue
@@ -514,13 +541,6 @@ __global__ void __launch_bounds__(kThreads)
 // then plan[0] = number of items, plan[1] = the work counter (zeroed here).
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 1024;  // item length in blocks, clamped; one bucket per thread
-
-__device__ __forceinline__ void griddep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 __device__ __forceinline__ void plan_counts(const int32_t* context_lens, int s,
                                             int max_context_len, int part_blocks, int& n,
@@ -848,6 +868,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
                            const int32_t* __restrict__ context_lens,
                            const int32_t* __restrict__ q_start, int num_seqs, int num_rows,
                            int num_q_heads, int max_context_len, int part_tokens, int max_parts) {
+  griddep_wait();  // the partials are complete
   reduce_rows_warp<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
                          num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x);
 }
@@ -863,6 +884,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
                       int num_q_heads, int max_context_len, int part_tokens, int max_parts,
                       int split_ctas) {
   extern __shared__ float s_w[];  // [max_parts] weights (split CTAs only)
+  griddep_wait();  // the partials are complete
   if ((int)blockIdx.x < split_ctas)
     reduce_rows_split<T, D>(out, part_o, part_lse, context_lens, q_start, num_seqs, num_rows,
                             num_q_heads, max_context_len, part_tokens, max_parts, blockIdx.x,
@@ -876,6 +898,24 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 template <typename T, int D>
 static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t stream);
 
+// Launch with programmatic stream serialization (the kernel itself waits for
+// its predecessor with griddep_wait before reading global memory).
+template <typename... Params, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <typename T, int D, bool kTwoRows, bool kMulti>
 static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
   using SM = DecodeSmem<D>;
@@ -883,12 +923,11 @@ static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((int64_t)a.max_parts * a.max_qtiles), a.num_kv_heads, a.num_seqs);
-  kern<<<grid, kThreads, SM::kAlloc, stream>>>(
-      a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, static_cast<const T*>(a.q),
-      a.q_start, a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride, a.context_lens,
-      a.num_q_heads, a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
-      a.max_parts, a.dev_error);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, grid, dim3(kThreads), SM::kAlloc, stream, a.tm_k, a.tm_v,
+                 static_cast<T*>(a.out), a.part_o, a.part_lse, static_cast<const T*>(a.q),
+                 a.q_start, a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride,
+                 a.context_lens, a.num_q_heads, a.group, a.num_blocks, a.max_context_len,
+                 a.scale_log2, a.part_blocks, a.max_parts, a.dev_error);
   if (e != cudaSuccess) return e;
   return launch_reduce_typed<T, D>(a, stream);
 }
@@ -902,10 +941,10 @@ static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t strea
   const int rows_per_cta = kReduceWarps * (32 / (D / 4));
   const int warp_ctas = (rows + rows_per_cta - 1) / rows_per_cta;
   if (a.max_parts <= kWarpRowMaxParts) {
-    lse_reduce_warp_kernel<T, D><<<warp_ctas, kReduceWarps * 32, 0, stream>>>(
-        static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start, a.num_seqs,
-        rows, a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts);
-    return cudaGetLastError();
+    return launch_pdl(lse_reduce_warp_kernel<T, D>, dim3(warp_ctas), dim3(kReduceWarps * 32), 0,
+                      stream, static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens,
+                      a.q_start, a.num_seqs, rows, a.num_q_heads, a.max_context_len,
+                      a.part_tokens, a.max_parts);
   }
   // Rows of more: a CTA each, one wave of CTAs striding over the rows.
   auto kern = lse_reduce_kernel<T, D>;
@@ -922,10 +961,10 @@ static cudaError_t launch_reduce_typed(const DecodeLaunch& a, cudaStream_t strea
   if (e != cudaSuccess) return e;
   const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
   const int split_ctas = (int)(rows < wave ? rows : wave);
-  kern<<<warp_ctas + split_ctas, kReduceWarps * 32, wbytes, stream>>>(
-      static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start, a.num_seqs, rows,
-      a.num_q_heads, a.max_context_len, a.part_tokens, a.max_parts, split_ctas);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(warp_ctas + split_ctas), dim3(kReduceWarps * 32), wbytes, stream,
+                    static_cast<T*>(a.out), a.part_o, a.part_lse, a.context_lens, a.q_start,
+                    a.num_seqs, rows, a.num_q_heads, a.max_context_len, a.part_tokens,
+                    a.max_parts, split_ctas);
 }
 
 template <typename T>
