@@ -510,23 +510,13 @@ __global__ void __launch_bounds__(kThreads)
                       max_context_len, scale_log2, part_blocks, max_parts,  dev_error};
   const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x;
   const int qtile = kMulti ? (int)(blockIdx.x / (unsigned)max_parts) : 0;
-  // Barriers and descriptor prefetch before the dependency wait: they touch
-  // no memory the previous kernel writes.
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < SM::kStages; ++s) mbar_init(&bars[warp * SM::kStages + s], 1);
-    fence_barrier_init();
-    if (warp == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-    }
-  }
-  __syncwarp();
+  // Launched as a programmatic dependent: the CTA is resident when the
+  // previous kernel ends, and waits for it before any read (empty
+  // partitions then exit before setting up barriers).
   griddep_wait();
   uint32_t ring = 0;
   (void)attend_item<T, D, kTwoRows, kMulti>(A, smem, bars, part, blockIdx.y, blockIdx.z, qtile,
-                                            false, ring);
+                                            true, ring);
 }
 
 // ---------------------------------------------------------------- work queue
