@@ -166,3 +166,38 @@ def test_full_size_skewed_sampled_rows():
     rng = np.random.default_rng(5)
     seqs = np.unique(np.concatenate([long_seqs, rng.choice(256, size=12, replace=False)]))
     _check(w, seqs=seqs)
+
+
+def test_plan_lists_every_item_once_longest_first():
+    """White-box check of the work list the plan kernel leaves in the
+    workspace (after pa_decode's partials: num_seqs * partitions 32-bit items
+    (seq << 16) | partition, then the item count): every non-empty partition
+    of every sequence exactly once (one item for an empty context), in
+    non-increasing order of its length in blocks."""
+    lens = [0, 5, 600, 1500, 40, 2100, 16, 17]
+    w = W.decode_workload("plan", lens, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                          dtype="bf16", seed=61)
+    d = DeviceStep(w).step()
+    S, P, Hq, D = len(lens), 512, 8, 128
+    max_ctx = w.max_context_len
+    ws = pa.alloc_workspace(S, Hq, D, max_ctx, P, "cuda", persistent=True)
+    ws.fill_(0xFF)
+    _persistent(d, ws=ws)
+    parts = -(-max_ctx // P)
+    base = pa.decode_workspace_size(S, Hq, D, max_ctx, P)
+    items_bytes = S * parts * 4
+    host = ws.cpu().numpy()
+    items = host[base:base + items_bytes].view(np.int32)
+    plan = host[base + (-(-items_bytes // 256)) * 256:][:8].view(np.int32)
+    pb = P // 16
+    want = {}
+    for s, L in enumerate(lens):
+        nblk = -(-L // 16)
+        n = max(1, -(-nblk // pb))
+        for p in range(n):
+            want[(s, p)] = min(pb, nblk - p * pb) if nblk else 0
+    assert int(plan[0]) == len(want)
+    got = [(int(v) >> 16, int(v) & 0xFFFF) for v in items[:len(want)]]
+    assert sorted(got) == sorted(want)
+    sizes = [want[i] for i in got]
+    assert all(a >= b for a, b in zip(sizes, sizes[1:])), sizes
