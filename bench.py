@@ -46,7 +46,8 @@ WORKLOAD_TEXT = {
     "long": "long-context 70B-shaped GQA decode, 1 layer: batch 8, H_q=64, H_kv=8, D=128, bf16, "
             "ctx U[32768,131072], split-K 512-token partitions + LSE reduce",
     "spec_verify": "speculative verify on the Llama-3-8B GQA batch: 256 seqs, 4 draft tokens each "
-                   "(causal in the chunk), H_q=32, H_kv=8, D=128, bf16, ctx lognormal(1024, 1)",
+                   "(causal in the chunk), H_q=32, H_kv=8, D=128, bf16, ctx lognormal(1024, 1), "
+                   "2048-token partitions",
     "chunked_prefill": "chunked prefill, Llama-3-8B shape: 16 prompts of U[1024,8192] tokens, "
                        "next 256-token chunk each, H_q=32, H_kv=8, D=128, bf16",
     "skewed": "skewed-length decode, Llama-3-8B GQA shape: batch 256, 4 contexts U[65536,131072] "

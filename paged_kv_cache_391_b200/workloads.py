@@ -277,12 +277,15 @@ def spec_verify(seed: int = 396, batch: int = 256, draft: int = 4) -> DecodeWork
     """Speculative-decoding verification on the Llama-3-8B-shaped GQA batch:
     each of 256 sequences (lognormal lengths, median 1024) checks ``draft``
     proposed tokens in one pass; with 4 query heads per KV head, 4 tokens fill
-    one 16-row tile."""
+    one 16-row tile. Split-K partitions of 2048 tokens: a partition's merge of
+    16 rows costs four times a decode tile's, so longer partitions pay it
+    less often (the 256 x 8 (sequence, KV head) pairs still fill the GPU)."""
     rng = np.random.default_rng(seed)
     lens = np.clip(np.round(np.exp(np.log(1024.0) + rng.standard_normal(batch))),
                    16, 8192).astype(np.int64)
     return chunk_workload("spec_verify", lens, np.full(batch, draft), num_q_heads=32,
-                          num_kv_heads=8, head_dim=128, dtype="bf16", seed=seed, rng=rng)
+                          num_kv_heads=8, head_dim=128, dtype="bf16", seed=seed, rng=rng,
+                          partition_tokens=2048)
 
 
 def chunked_prefill(seed: int = 397, batch: int = 16, chunk: int = 256) -> DecodeWorkload:
