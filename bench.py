@@ -52,7 +52,7 @@ WORKLOAD_TEXT = {
                        "next 256-token chunk each, H_q=32, H_kv=8, D=128, bf16",
     "skewed": "skewed-length decode, Llama-3-8B GQA shape: batch 256, 4 contexts U[65536,131072] "
               "among 252 lognormal(median 512, sigma 0.7) clipped [16,4096], H_q=32, H_kv=8, "
-              "D=128, bf16",
+              "D=128, bf16, 2048-token partitions",
 }
 
 

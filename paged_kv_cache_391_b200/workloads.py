@@ -404,14 +404,17 @@ def skewed(seed: int = 398, batch: int = 256, n_long: int = 4, long_lo: int = 65
     uniform in [65536, 131072] tokens among short ones, lognormal with median
     512 (sigma 0.7) clipped to [16, 4096]; the long ones sit at random batch
     positions. max_context_len is set by the longest, so a grid sized by it
-    holds mostly empty partitions: the case a work-queue schedule is for."""
+    holds mostly empty partitions: the case a work-queue schedule is for.
+    Split-K partitions of 2048 tokens (the long rows then reduce 56
+    partitions, not 223)."""
     rng = np.random.default_rng(seed)
     lens = np.clip(np.round(np.exp(np.log(short_median) + sigma * rng.standard_normal(batch))),
                    16, short_hi).astype(np.int64)
     where = rng.choice(batch, size=n_long, replace=False)
     lens[where] = rng.integers(long_lo, long_hi, size=n_long, endpoint=True)
     return decode_workload("skewed", lens, num_q_heads=32, num_kv_heads=8, head_dim=128,
-                           dtype="bf16", seed=seed, pool_factor=1.25, rng=rng)
+                           dtype="bf16", seed=seed, pool_factor=1.25, rng=rng,
+                           partition_tokens=2048)
 
 
 CONFIGS = {
