@@ -178,7 +178,13 @@ pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
  * "Chunked Prefill: Don't Let Long Prompts Consume the Entire Budget") and of
  * verifying speculative draft tokens ("The Memory Wall ...", "The Next
  * Frontier: Speculative Decoding and Beyond"). With one token per sequence it
- * equals pa_decode.
+ * equals pa_decode bit for bit.
+ * Two implementations, chosen per call: when max_query_len * group_size >= 64,
+ * head_dim is 128, group_size is a power of two and partition_tokens is 0 or a
+ * multiple of 64, the chunk runs on the tcgen05 tensor cores (accumulators in
+ * tensor memory, one CTA per pair of 128-row query tiles); otherwise on the
+ * 16-row mma.sync tiles of pa_decode. Both are within the same tolerance of
+ * the exact result; they are not bitwise equal to each other.
  *   out, q          device, [num_q_tokens][num_q_heads][head_dim]
  *   q_start         device int32 [num_seqs + 1], non-decreasing, q_start[0] = 0
  *   max_query_len   host upper bound of Tq (sizes the launch); Tq must also be
