@@ -1,7 +1,8 @@
 /*
  * pa.h -- C ABI of libpa: the paged-KV-cache decode hot path on B200 (sm_100a).
  *
- * Three operations of PagedAttention decode, as the pages describe them:
+ * The operations of PagedAttention's decode path, as the pages describe them
+ * (the first three are the hot path; the rest follow below):
  *
  *   pa_write_kv     store this step's new K/V rows in their cache slots
  *                   ("Optimizing LLM Inference: From PagedAttention to AI
@@ -21,6 +22,13 @@
  *                   copy-on-write ("Optimizing LLM Inference ...",
  *                   "Copy-on-Write"; "PagedAttention", "KV Cache Sharing
  *                   (Copy-on-Write)").
+ *   pa_decode_persistent  pa_decode scheduled as a device-planned work queue.
+ *   pa_prefill_chunk      attention of several query tokens per sequence
+ *                         (chunked prefill, speculative verification).
+ *   pa_swap_blocks        blocks between a device pool and a pinned host pool.
+ *   pa_bm_*               host block manager: refcounted blocks, on-demand
+ *                         allocation, copy-on-write decisions.
+ *   pa_decode_static      pa_decode with a scratch array compiled into libpa.
  *
  * Memory layout (all device memory, row-major, no padding):
  *   k_cache, v_cache : [num_blocks][num_kv_heads][PA_BLOCK_SIZE][head_dim]
@@ -39,8 +47,10 @@
  * Ownership: the caller allocates and owns every buffer, the workspace and the
  * stream. The library borrows the pointers for the duration of the
  * asynchronous call, allocates no device memory, keeps no per-call state and
- * never synchronises the stream. Every call is stream-ordered on `stream`
- * (a cudaStream_t; NULL is the legacy default stream).
+ * never synchronises the stream (exceptions, each documented below: the
+ * scratch array of pa_decode_static and the host object a pa_bm handle owns).
+ * Every call is stream-ordered on `stream` (a cudaStream_t; NULL is the legacy
+ * default stream).
  *
  * Errors: problems visible on the host (a NULL pointer, an unsupported shape,
  * a too-small workspace, an out-of-range argument) return a status and launch
