@@ -33,3 +33,43 @@ def test_l2_notes():
 def test_cpu_leg_on_tiny():
     r = bench.oracle_sample(W.tiny(), 0.05)
     assert r["gbs"] > 0 and r["cores"] >= 1 and "rows" in r["sample"]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints
+    one JSON line with the keys the driver reads, on a bounded sample."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "2", "--warmup", "1",
+                        "--cpu-seconds", "0.2"], capture_output=True, text=True, timeout=300,
+                       cwd=root)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"] == d["e2e"]["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_recorded_traffic_follows_the_kernel_sources():
+    """A traffic figure is reported for a full-size workload only while the
+    hash of its kernel family's sources matches the recorded one."""
+    assert bench.recorded_traffic("mha", batch=16) is None        # not the full size
+    assert bench.recorded_traffic("no_such_workload", None) is None
+    fam = {"chunked_prefill": "tcgen05", "mha": "mma"}
+    with open(bench.TRAFFIC_FILE) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for key, h, nbytes, alg, ratio in rows:
+        workload, _, sched = key.partition(":")
+        want = bench.kernel_source_hash("tcgen05" if workload in bench.TC_WORKLOADS else "mma")
+        got = bench.recorded_traffic(workload, None, sched or "grid")
+        assert got == (int(nbytes) if h == want else None), key
+        assert abs(int(nbytes) / int(alg) - float(ratio)) < 1e-3
+    assert set(fam) <= {r[0].partition(":")[0] for r in rows}
