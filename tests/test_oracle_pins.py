@@ -464,3 +464,23 @@ def test_one_token_chunks_are_decode():
     a = oracle.prefill_chunk(q, q_start, kp, vp, bt, cl, 0.125, "bf16")
     b = oracle.decode(q, kp, vp, bt, cl, 0.125, "bf16")
     assert np.array_equal(a, b)
+
+
+def test_prefill_chunk_scale_zero_is_the_running_mean_of_values():
+    """Closed form: with scale 0 every visible key weighs the same, so query
+    token t of a chunk of Tq at the end of an L-token context returns the mean
+    of V over positions 0 .. L-Tq+t (a prefix mean that grows by one key per
+    query token)."""
+    rng = np.random.default_rng(77)
+    lens, tq, Hq, Hkv, D = [12, 33], [5, 33], 4, 2, 64
+    q, ck, cv, kp, vp, bt, cl = _random_case(rng, lens, Hq, Hkv, D, "f16")
+    q_start = np.concatenate([[0], np.cumsum(tq)]).astype(np.int32)
+    qc = _bits(rng, (int(q_start[-1]), Hq, D), "f16")
+    out = oracle.prefill_chunk(qc, q_start, kp, vp, bt, cl, 0.0, "f16")
+    for s, (L, T) in enumerate(zip(lens, tq)):
+        V = oracle.decode16(cv[s], "f16")                   # [L, Hkv, D]
+        for t in range(T):
+            n = L - T + t + 1
+            mean = V[:n].mean(axis=0)                       # [Hkv, D]
+            want = np.repeat(mean, Hq // Hkv, axis=0)       # query head h -> KV head h // g
+            np.testing.assert_allclose(out[q_start[s] + t], want, rtol=1e-12, atol=1e-13)
