@@ -166,3 +166,31 @@ def _decode_persistent(L, **kw):
 ])
 def test_decode_persistent_rejects_on_the_host(L, kw, status):
     assert _decode_persistent(L, **kw) == status
+
+
+def _prefill(L, **kw):
+    a = dict(out=FAKE, q=FAKE, qs=FAKE, nq=8, maxq=4, k=FAKE, v=FAKE, bt=FAKE, stride=4, cl=FAKE,
+             S=2, Hq=8, g=4, D=128, bs=16, NB=10, max_ctx=64, scale=0.1, P=512, ws=None,
+             ws_bytes=0, err=None, dt=1)
+    a.update(kw)
+    return L.pa_prefill_chunk(a["out"], a["q"], a["qs"], a["nq"], a["maxq"], a["k"], a["v"],
+                              a["bt"], a["stride"], a["cl"], a["S"], a["Hq"], a["g"], a["D"],
+                              a["bs"], a["NB"], a["max_ctx"], ctypes.c_float(a["scale"]), a["P"],
+                              a["ws"], a["ws_bytes"], a["err"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qs=None), pa.PA_ERR_INVALID_ARG),                  # q_start is required
+    (dict(qs=FAKE + 2), pa.PA_ERR_INVALID_ARG),              # misaligned q_start
+    (dict(maxq=-1), pa.PA_ERR_INVALID_ARG),
+    (dict(nq=-1), pa.PA_ERR_INVALID_ARG),
+    (dict(g=3), pa.PA_ERR_UNSUPPORTED),
+    (dict(D=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(P=100), pa.PA_ERR_UNSUPPORTED),                    # not a multiple of 16
+    (dict(max_ctx=2048, stride=128), pa.PA_ERR_INVALID_ARG),  # needs a workspace
+    (dict(max_ctx=2048, stride=128, ws=FAKE, ws_bytes=100), pa.PA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(nq=0), pa.PA_OK),                                  # no query rows: nothing to do
+    (dict(S=0), pa.PA_OK),
+])
+def test_prefill_chunk_rejects_on_the_host(L, kw, status):
+    assert _prefill(L, **kw) == status
