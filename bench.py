@@ -61,7 +61,12 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mha", choices=list(WORKLOAD_TEXT))
+    ap.add_argument("--workload", default="long", choices=list(WORKLOAD_TEXT),
+                    help="the headline workload (default: the long-context config, the "
+                         "largest that fits one GPU)")
+    ap.add_argument("--also", default="gqa",
+                    help="comma-separated workloads measured in the same run and reported "
+                         "under 'also' (empty: none)")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling only)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--op", default="step", choices=["step", "swap", "blockmgr"],
@@ -72,8 +77,9 @@ def parse():
                     help="decode schedule: grid = pa_decode (one CTA per partition); "
                          "persistent = pa_decode_persistent (plan + work queue)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--event-stride", type=int, default=4,
-                    help="time the attention call with events on every kth timed step")
+    ap.add_argument("--op-seconds", type=float, default=0.6,
+                    help="target GPU time of each per-operation timing loop")
+    ap.add_argument("--no-read-probe", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle sample")
@@ -177,7 +183,8 @@ class ClockSampler:
         "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
     }
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_s: float = 0.001):
+        self.interval = interval_s
         self.samples, self.reasons, self.err = [], set(), None
         self.max_mhz = None
         self._stop = threading.Event()
@@ -206,7 +213,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception as e:
                 self.err = str(e)
-            time.sleep(0.005)
+            time.sleep(self.interval)
 
     def __enter__(self):
         if self.nv:
@@ -223,8 +230,11 @@ class ClockSampler:
         if not self.nv:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_min_mhz": min(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+                "samples": len(self.samples),
+                "how": f"NVML every {self.interval * 1e3:g} ms across every timed loop (the K "
+                       f"steps, the per-operation loops, the read-ceiling probe, e2e)"}
 
 
 # --------------------------------------------------------------------------- CPU (oracle) leg
@@ -316,11 +326,103 @@ class PackedInputs:
         return out
 
 
-def run_gpu(args, rank, world, device):
+def spare_blocks(w) -> np.ndarray:
+    """Physical blocks no table reaches and no copy reads or writes: targets
+    for timing block copies without disturbing the step's cache."""
+    used = np.zeros(w.num_blocks, dtype=bool)
+    for s, L in enumerate(w.context_lens):
+        n = -(-int(L) // w.block_size)
+        used[w.block_tables[s, :n]] = True
+    for pairs in (w.copy_pairs, np.asarray(w.notes.get("fork_pairs", []), np.int64).reshape(-1, 2)):
+        if len(pairs):
+            used[pairs.reshape(-1)] = True
+    return np.flatnonzero(~used)
+
+
+def timing_copy_pairs(w):
+    """The block copies timed on their own, and what they are: the config's
+    copy-on-write forks when it has any (into spare blocks when the fork
+    happened before the step), else a fork of every sequence's last block
+    into a spare block (the cost of forking each sequence once)."""
+    spare = spare_blocks(w)
+    if len(w.copy_pairs):
+        return w.copy_pairs, "the step's copy-on-write forks"
+    forks = np.asarray(w.notes.get("fork_pairs", []), np.int64).reshape(-1, 2)
+    if len(forks):
+        n = min(len(forks), len(spare))
+        return (np.stack([forks[:n, 0], spare[:n]], axis=1).astype(np.int64),
+                f"the config's {n} copy-on-write forks of the partial prefix block "
+                f"(made before the step; timed into spare blocks)")
+    last = np.array([w.block_tables[s, max(0, -(-int(L) // w.block_size) - 1)]
+                     for s, L in enumerate(w.context_lens)], np.int64)
+    n = min(len(last), len(spare))
+    return (np.stack([last[:n], spare[:n]], axis=1).astype(np.int64),
+            f"a fork of each of {n} sequences' last block into a spare block "
+            f"(the config's step copies nothing)")
+
+
+def waste_stats(w) -> dict:
+    """Slots allocated but not holding a token: the unused tail of each
+    sequence's last block (the only waste of 16-token paging)."""
+    L = w.context_lens.astype(np.int64)
+    alloc = -(-L // w.block_size) * w.block_size
+    waste = alloc - L
+    return {"mean_slots_per_seq": round(float(waste.mean()), 3),
+            "pct_of_allocated_slots": round(100.0 * float(waste.sum()) / float(alloc.sum()), 4)}
+
+
+def read_ceiling(device, nbytes: int = 2 << 30, reps: int = 10) -> dict:
+    """The GPU's streaming-read ceiling (pa_read_probe, both methods): best of
+    `reps` timed passes over a buffer of `nbytes` (16x the L2)."""
+    import torch
+    from paged_kv_cache_391_b200 import pa
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    sink = torch.zeros(1, dtype=torch.int64, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    out = {"bytes": nbytes}
+    for method, name in ((0, "vector_loads_gbs"), (1, "bulk_copies_gbs")):
+        for _ in range(3):
+            pa.read_probe(buf, sink, method=method, dev_error=err)
+        best = None
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            pa.read_probe(buf, sink, method=method, dev_error=err)
+            b.record()
+            b.synchronize()
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+        out[name] = round(nbytes / (best / 1e3) / 1e9, 1)
+    out["gbs"] = max(out["vector_loads_gbs"], out["bulk_copies_gbs"])
+    out["device_errors"] = int(err.item())
+    del buf
+    return out
+
+
+def time_loop(fn, reps: int, stream, blocker=None) -> float:
+    """Average ms per call of `reps` back-to-back calls of fn on `stream`,
+    timed by events at the two ends of the loop. For calls shorter than their
+    host-side launch, `blocker` first queues enough GPU work that every call
+    is queued before the GPU reaches the first event."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if blocker is not None:
+        blocker()
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_gpu(args, name, rank, world, device, probe_buf=None, e2e_on=True):
+    """One workload on this rank: the K-step timed region, then each
+    operation of the step in its own loop, then the end-to-end run."""
     import torch
     from paged_kv_cache_391_b200 import pa
 
-    w = make_workload(args.workload, args.batch, seed_offset=rank)
+    w = make_workload(name, args.batch if name == args.workload else None, seed_offset=rank)
     if args.partition_tokens is not None:
         w.partition_tokens = args.partition_tokens
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
@@ -346,16 +448,20 @@ def run_gpu(args, rank, world, device):
     max_parts = 1 if (P == 0 or max_ctx <= P) else -(-max_ctx // P)
     launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + \
         1 + (1 if max_parts > 1 else 0) + (1 if persistent else 0)
+    copy_pairs_t, copy_what = timing_copy_pairs(w)
+    copy_pairs_dev = torch.from_numpy(copy_pairs_t).to(device)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def step(x, o, e_dec=None):
+    def copies(x):
         if x["pairs"].numel():
             pa.copy_blocks([k_cache], [v_cache], x["pairs"], dev_error=err, stream=stream)
+
+    def write(x):
         pa.write_kv(x["new_k"], x["new_v"], k_cache, v_cache, x["slots"], dev_error=err,
                     stream=stream)
-        if e_dec is not None:
-            e_dec[0].record(stream)
+
+    def attend(x, o):
         if "q_start" in x:
             pa.prefill_chunk(o, x["q"], x["q_start"], k_cache, v_cache, x["bt"], x["cl"],
                              scale=w.scale, max_query_len=max_q, max_context_len=max_ctx,
@@ -364,8 +470,11 @@ def run_gpu(args, rank, world, device):
             pa.decode(o, x["q"], k_cache, v_cache, x["bt"], x["cl"], scale=w.scale,
                       max_context_len=max_ctx, partition_tokens=P, workspace=ws, dev_error=err,
                       stream=stream, persistent=persistent)
-        if e_dec is not None:
-            e_dec[1].record(stream)
+
+    def step(x, o):
+        copies(x)
+        write(x)
+        attend(x, o)
 
     def barrier():
         if world > 1:
@@ -376,22 +485,40 @@ def run_gpu(args, rank, world, device):
     for _ in range(args.warmup):
         step(inp, out)
     barrier()
-    # The attention call's own duration is taken with events around it on
-    # every kth timed step only: an event between the KV write and the
-    # partition kernel stops the latter's programmatic early launch, so
-    # bracketing every step would slow the loop whose throughput is `value`.
-    stride = max(1, args.event_stride)
-    dec_events = [(ev(), ev()) for _ in range(0, args.steps, stride)]
     t_start, t_end = ev(), ev()
-    with ClockSampler(device.index if device.index is not None else 0) as clocks:
-        barrier()
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(inp, out, dec_events[i // stride] if i % stride == 0 else None)
-        t_end.record(stream)
-        barrier()
+    barrier()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(inp, out)
+    t_end.record(stream)
+    barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in dec_events]))
+
+    # ---- each operation of the step in its own loop (events at the loop ends only)
+    step_ms = elapsed_ms / max(1, args.steps)
+    sink = torch.zeros(1, dtype=torch.int64, device=device)
+
+    def blocker():  # ~10 ms of queued GPU work ahead of a loop of short calls
+        if probe_buf is None:
+            return
+        for _ in range(30):
+            pa.read_probe(probe_buf, sink, method=0, stream=stream)
+
+    att_reps = int(min(20000, max(20, args.op_seconds / max(step_ms, 1e-3) * 1e3)))
+    for _ in range(3):
+        attend(inp, out)
+    att_ms = time_loop(lambda: attend(inp, out), att_reps, stream)
+    short_reps = 200
+    rounds = max(1, int(args.op_seconds / 0.012))
+    write_ms = min(time_loop(lambda: write(inp), short_reps, stream, blocker)
+                   for _ in range(rounds)) if len(w.slot_mapping) else None
+    copy_ms = min(time_loop(lambda: pa.copy_blocks([k_cache], [v_cache], copy_pairs_dev,
+                                                   dev_error=err, stream=stream),
+                            short_reps, stream, blocker)
+                  for _ in range(rounds)) if len(copy_pairs_t) else None
+    # restore the step's cache state (the copy loop may write over forked blocks)
+    step(inp, out)
+    torch.cuda.synchronize(device)
     errors = int(err.item())
 
     # ---- e2e: every step uploads its packed inputs from pinned host memory
@@ -399,7 +526,7 @@ def run_gpu(args, rank, world, device):
     # a download stream let step i+1's upload and step i's download overlap
     # step i's kernels.
     e2e = None
-    if not args.no_e2e:
+    if e2e_on and not args.no_e2e:
         up_stream, down_stream = torch.cuda.Stream(device), torch.cuda.Stream(device)
         dev_in = [torch.empty(packed.nbytes, dtype=torch.uint8, device=device) for _ in range(2)]
         views = [packed.views(b) for b in dev_in]
@@ -441,7 +568,11 @@ def run_gpu(args, rank, world, device):
         barrier()
         e2e = {"ms": a.elapsed_time(b), "h2d": packed.payload,
                "d2h": host_out[0].numel() * host_out[0].element_size()}
-    return w, elapsed_ms, dec_ms, errors, clocks.report(), e2e, launches_per_step
+    return {"w": w, "elapsed_ms": elapsed_ms, "att_ms": att_ms, "att_reps": att_reps,
+            "write_ms": write_ms, "copy_ms": copy_ms, "copy_pairs": int(len(copy_pairs_t)),
+            "copy_what": copy_what, "short_reps": short_reps, "rounds": rounds,
+            "errors": errors, "e2e": e2e, "launches": launches_per_step,
+            "persistent": persistent}
 
 
 def l2_note(w) -> str:
@@ -457,20 +588,26 @@ def l2_note(w) -> str:
     return f"KV per step {kv / 1e6:.0f} MB is within 2x of the {L2_BYTES / 1e6:.0f} MB L2"
 
 
-def reduce_over_ranks(elapsed_ms, e2e_ms, kv_bytes, seqs, errors, world, device=None):
-    """Whole-job figures: the slowest rank's times (max) and every rank's work
-    (sum). One all_reduce each; every rank takes the same collective steps."""
-    if world <= 1:
-        return {"ms": float(elapsed_ms), "e2e_ms": float(e2e_ms), "kv": float(kv_bytes),
-                "seqs": float(seqs), "errors": int(errors)}
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    s = torch.tensor([kv_bytes, seqs, errors], dtype=torch.float64, device=device)
-    dist.all_reduce(s, op=dist.ReduceOp.SUM)
-    return {"ms": float(t[0]), "e2e_ms": float(t[1]), "kv": float(s[0]), "seqs": float(s[1]),
-            "errors": int(s[2])}
+def reduce_over_ranks(res, world, device=None):
+    """Whole-job figures of one workload: the slowest rank's times (max) and
+    every rank's work (sum). One all_reduce each; every rank takes the same
+    collective steps."""
+    w = res["w"]
+    times = [res["elapsed_ms"], res["e2e"]["ms"] if res["e2e"] else 0.0, res["att_ms"],
+             res["write_ms"] or 0.0, res["copy_ms"] or 0.0]
+    work = [float(w.kv_bytes()), float(w.num_seqs), float(res["errors"])]
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor(times, dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        s = torch.tensor(work, dtype=torch.float64, device=device)
+        dist.all_reduce(s, op=dist.ReduceOp.SUM)
+        times, work = t.tolist(), s.tolist()
+    return {"ms": float(times[0]), "e2e_ms": float(times[1]), "att_ms": float(times[2]),
+            "write_ms": float(times[3]) if res["write_ms"] is not None else None,
+            "copy_ms": float(times[4]) if res["copy_ms"] is not None else None,
+            "kv": float(work[0]), "seqs": float(work[1]), "errors": int(work[2])}
 
 
 def run_swap(args, device):
@@ -584,6 +721,108 @@ def run_blockmgr(args):
     return 0
 
 
+def kernel_name(w, args) -> str:
+    if w.q_start is not None:
+        return ("pa_prefill_chunk (prefill_tc_kernel on tcgen05 + lse_reduce_kernel)"
+                if int(np.diff(w.q_start).max()) * w.group_size >= 64 else
+                "pa_prefill_chunk (decode_partition_kernel + lse_reduce_kernel)")
+    if args.scheduler == "persistent":
+        return ("pa_decode_persistent (decode_plan_kernel + decode_persistent_kernel + "
+                "lse_reduce_kernel)")
+    return "pa_decode (decode_partition_kernel + lse_reduce_kernel)"
+
+
+def workload_record(name, res, agg, args, world, ceiling) -> dict:
+    """The figures of one workload: step throughput, the attention call
+    against its roofline, each operation's own time, end to end."""
+    w = res["w"]
+    K = args.steps
+    peak, peak_src = measured_peaks()
+    tpeak, tpeak_src = measured_tensor_peak()
+    sb = w.step_bytes()
+    elapsed_ms = agg["ms"]
+    att_ms = agg["att_ms"]
+    value = agg["kv"] * K / (elapsed_ms / 1e3) / 1e9
+    dec_achieved = sb["decode"] / (att_ms / 1e3) / 1e9
+    flops = attention_flops(w)
+    tensor_bound = flops / (tpeak * 1e12) > sb["decode"] / (peak * 1e9)
+    tflops = flops / (att_ms / 1e3) / 1e12
+    traffic = recorded_traffic(name, args.batch if name == args.workload else None,
+                               args.scheduler)
+    roof = {
+        "kernel": kernel_name(w, args),
+        "bound": "tensor" if tensor_bound else "hbm",
+        "achieved": round(tflops, 2) if tensor_bound else round(dec_achieved, 1),
+        "peak": tpeak if tensor_bound else peak,
+        "peak_source": tpeak_src if tensor_bound else peak_src,
+        "unit": "TFLOP/s" if tensor_bound else "GB/s",
+        "frac": round(tflops / tpeak, 4) if tensor_bound else round(dec_achieved / peak, 4),
+        "kv_gbs": round(dec_achieved, 1),
+        "tflops": round(tflops, 2),
+        "flops_per_launch": flops,
+        "algorithmic_bytes_per_launch": sb["decode"],
+        "timing": f"CUDA events at the two ends of a loop of {res['att_reps']} back-to-back "
+                  f"attention calls on the launching stream (after the {K}-step timed region; "
+                  f"max over ranks)",
+        "traffic": traffic,
+        "traffic_ratio": round(traffic / sb["decode"], 4) if traffic else None,
+        "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the call's "
+                        "kernels per call (profiles/dram_traffic.txt; scaled from a reduced "
+                        "batch where noted there; null if a kernel source changed since)",
+    }
+    if ceiling and not tensor_bound:
+        roof["peak_read"] = ceiling["gbs"]
+        roof["frac_read"] = round(dec_achieved / ceiling["gbs"], 4)
+        roof["peak_read_source"] = ("pa_read_probe in this run: best of 10 passes over "
+                                    f"{ceiling['bytes'] >> 30} GiB, max of vector loads "
+                                    f"({ceiling['vector_loads_gbs']}) and bulk copies "
+                                    f"({ceiling['bulk_copies_gbs']}) GB/s")
+    if traffic and not tensor_bound:
+        roof["dram_gbs"] = round(traffic / (att_ms / 1e3) / 1e9, 1)
+    rec = {
+        "value": round(value, 2), "unit": "GB/s", "ms_per_step": round(elapsed_ms / K, 5),
+        "seq_steps_per_s": round(agg["seqs"] * K / (elapsed_ms / 1e3), 1),
+        "hbm_frac_of_peak": round(value / peak, 4),
+        "dtype": w.dtype,
+        "config": {
+            "workload": WORKLOAD_TEXT[name] + (f" [batch overridden to {args.batch}]"
+                                               if args.batch is not None and name == args.workload
+                                               else ""),
+            "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": 16, "partition_tokens": w.partition_tokens,
+            "mean_context_len": float(np.mean(w.context_lens)),
+            "kv_bytes_per_step": w.kv_bytes(),
+            "step": ("copy_blocks + write_kv + attention" if len(w.copy_pairs)
+                     else "write_kv + attention") + " (partitions + LSE reduce when split)",
+            "scheduler": ("persistent: plan kernel + work-queue grid of SMs x resident CTAs"
+                          if res["persistent"] else
+                          "grid: one CTA per (partition, KV head, sequence)"),
+            "accumulate": "fp32",
+            "l2": l2_note(w),
+            "last_block_waste": waste_stats(w),
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+        },
+        "roofline": roof,
+        "sub_ms": {"attention": round(att_ms, 5),
+                   "write_kv": None if agg["write_ms"] is None else round(agg["write_ms"], 5),
+                   "copy_blocks": None if agg["copy_ms"] is None else round(agg["copy_ms"], 5)},
+        "op_us": {"write_kv": None if agg["write_ms"] is None else round(agg["write_ms"] * 1e3, 2),
+                  "copy_blocks": None if agg["copy_ms"] is None else round(agg["copy_ms"] * 1e3, 2),
+                  "copy_blocks_pairs": res["copy_pairs"], "copy_blocks_what": res["copy_what"],
+                  "timing": f"each op alone, {res['short_reps']} back-to-back calls queued "
+                            f"behind GPU work, events at the loop ends; best of "
+                            f"{res['rounds']} loops"},
+        "gpu_launches": res["launches"] * K,
+        "device_errors": agg["errors"],
+    }
+    if res["e2e"]:
+        e = res["e2e"]
+        rec["e2e"] = {"value": round(agg["kv"] * K / (agg["e2e_ms"] / 1e3) / 1e9, 2),
+                      "unit": "GB/s", "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                      "ms_per_step": round(agg["e2e_ms"] / K, 5)}
+    return rec
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -609,94 +848,54 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
 
-    w, elapsed_ms, dec_ms, errors, clocks, e2e, launches = run_gpu(args, rank, world, device)
-
-    kv_bytes = w.kv_bytes()
-    sb = w.step_bytes()
-    seqs = w.num_seqs
-    agg = reduce_over_ranks(elapsed_ms, e2e["ms"] if e2e else 0.0, kv_bytes, seqs, errors,
-                            world, device)
-    elapsed_ms, kv_total, seqs_total, errors = agg["ms"], agg["kv"], agg["seqs"], agg["errors"]
-    if e2e:
-        e2e["ms"] = agg["e2e_ms"]
-
-    peak, peak_src = measured_peaks()
-    tpeak, tpeak_src = measured_tensor_peak()
-    K = args.steps
-    value = kv_total * K / (elapsed_ms / 1e3) / 1e9
-    dec_achieved = sb["decode"] / (dec_ms / 1e3) / 1e9
-    flops = attention_flops(w)
-    tensor_bound = flops / (tpeak * 1e12) > sb["decode"] / (peak * 1e9)
+    names = [args.workload] + [n for n in args.also.split(",") if n and n != args.workload]
+    for n in names:
+        if n not in WORKLOAD_TEXT:
+            raise SystemExit(f"unknown workload {n}")
+    records = {}
+    ceiling = None
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        # a buffer 16x the L2: the read-ceiling probe's input, and the GPU work
+        # queued ahead of the loops of short calls
+        probe_buf = torch.empty(2 << 30, dtype=torch.uint8, device=device)
+        if not args.no_read_probe:
+            ceiling = read_ceiling(device)
+        for i, name in enumerate(names):
+            res = run_gpu(args, name, rank, world, device, probe_buf=probe_buf)
+            agg = reduce_over_ranks(res, world, device)
+            records[name] = (res, agg)
+            if i + 1 < len(names):     # free this workload's pools before the next
+                res["w"] = _light(res["w"])
+                torch.cuda.empty_cache()
+        del probe_buf
+    head_res, head_agg = records[args.workload]
+    rec = workload_record(args.workload, head_res, head_agg, args, world, ceiling)
     line = {
         "metric": METRIC,
-        "value": round(value, 2),
+        "value": rec["value"],
         "unit": "GB/s",
         "n_gpus": world,
-        "steps": K,
+        "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(elapsed_ms / K, 5),
+        "ms_per_step": rec["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": w.dtype,
+        "dtype": rec["dtype"],
         "data": "synthetic (seeded N(0,1) q/K/V, seeded random block placement)",
-        "config": {
-            "workload": WORKLOAD_TEXT[args.workload] if args.batch is None
-            else WORKLOAD_TEXT[args.workload] + f" [batch overridden to {args.batch}]",
-            "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
-            "head_dim": w.head_dim, "block_size": 16, "partition_tokens": w.partition_tokens,
-            "mean_context_len": float(np.mean(w.context_lens)),
-            "kv_bytes_per_step": kv_bytes,
-            "step": "copy_blocks (if forks) + write_kv + decode (partitions + LSE reduce)",
-            "scheduler": ("persistent: plan kernel + work-queue grid of SMs x resident CTAs"
-                          if args.scheduler == "persistent" and w.q_start is None
-                          else "grid: one CTA per (partition, KV head, sequence)"),
-            "accumulate": "fp32",
-            "l2": l2_note(w),
-            "parallelism": f"dp{world} (independent sequences per GPU)",
-        },
-        "seq_steps_per_s": round(seqs_total * K / (elapsed_ms / 1e3), 1),
-        "hbm_frac_of_peak": round(value / peak, 4),
-        "roofline": {
-            "kernel": (("pa_prefill_chunk (prefill_tc_kernel on tcgen05 + lse_reduce_kernel)"
-                        if int(np.diff(w.q_start).max()) * w.group_size >= 64 else
-                        "pa_prefill_chunk (decode_partition_kernel + lse_reduce_kernel)")
-                       if w.q_start is not None else
-                       "pa_decode_persistent (decode_plan_kernel + decode_persistent_kernel + "
-                       "lse_reduce_kernel)" if args.scheduler == "persistent" else
-                       "pa_decode (decode_partition_kernel + lse_reduce_kernel)"),
-            "bound": "tensor" if tensor_bound else "hbm",
-            "achieved": round(flops / (dec_ms / 1e3) / 1e12, 2) if tensor_bound
-            else round(dec_achieved, 1),
-            "peak": tpeak if tensor_bound else peak,
-            "peak_source": tpeak_src if tensor_bound else peak_src,
-            "unit": "TFLOP/s" if tensor_bound else "GB/s",
-            "frac": round(flops / (dec_ms / 1e3) / 1e12 / tpeak, 4) if tensor_bound
-            else round(dec_achieved / peak, 4),
-            "kv_gbs": round(dec_achieved, 1),
-            "tflops": round(flops / (dec_ms / 1e3) / 1e12, 2),
-            "flops_per_launch": flops,
-            "algorithmic_bytes_per_launch": sb["decode"],
-            "timing": f"CUDA events around the attention call on every "
-                      f"{max(1, args.event_stride)}th of the {K} timed steps",
-            "traffic": recorded_traffic(args.workload, args.batch, args.scheduler),
-            "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
-                            "call's kernels (partition or persistent kernel, plan, LSE "
-                            "reduce) per call, full-size workload (profiles/dram_traffic.txt; "
-                            "null if a kernel source changed since)",
-        },
-        "sub_ms": {"decode": round(dec_ms, 5),
-                   "write_kv_and_copies": round(elapsed_ms / K - dec_ms, 5)},
-        "clocks": clocks,
-        "gpu_launches": launches * K,
-        "device_errors": errors,
     }
-    if e2e:
-        line["e2e"] = {"value": round(kv_total * K / (e2e["ms"] / 1e3) / 1e9, 2), "unit": "GB/s",
-                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": round(e2e["ms"] / K, 5)}
+    line.update({k: v for k, v in rec.items() if k not in line})
+    line["clocks"] = clocks.report()
+    if ceiling:
+        line["read_ceiling"] = ceiling
+    also = {}
+    for name in names[1:]:
+        r = workload_record(name, *records[name], args, world, ceiling)
+        also[name] = r
+    if also:
+        line["also"] = also
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample(w, args.cpu_seconds)
+        cb = oracle_sample(head_res["w"], args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(cb["gbs"], 4), "unit": "GB/s", "cores": cb["cores"],
                                 "kind": "oracle", "sample": cb["sample"],
                                 "seq_steps_per_s": round(cb["seq_steps_per_s"], 3),
@@ -708,6 +907,12 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _light(w):
+    """A workload without its cache pools (enough for the report)."""
+    import dataclasses
+    return dataclasses.replace(w, k_pool=w.k_pool[:1], v_pool=w.v_pool[:1])
 
 
 def main_reference(args, rank, world):

@@ -29,6 +29,7 @@
  *   pa_bm_*               host block manager: refcounted blocks, on-demand
  *                         allocation, copy-on-write decisions.
  *   pa_decode_static      pa_decode with a scratch array compiled into libpa.
+ *   pa_read_probe         measurement utility: the streaming-read ceiling.
  *
  * Memory layout (all device memory, row-major, no padding):
  *   k_cache, v_cache : [num_blocks][num_kv_heads][PA_BLOCK_SIZE][head_dim]
@@ -274,7 +275,10 @@ pa_status pa_swap_blocks(void* const* src_k, void* const* src_v, void* const* ds
  *     nothing (use pa_decode with a caller workspace for those).
  *   - The first call on a device looks the array's address up on that device
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture on the device.
+ *     before any stream capture on the device. The address is kept with the
+ *     id of the device's CUDA context; after cudaDeviceReset (a new context,
+ *     the library's device code loaded again) the next call looks it up
+ *     again, and that call too should precede any stream capture.
  *   - All calls on a device share the array. Nothing in it needs to start at
  *     zero, but calls whose kernels overlap on the GPU race on it: order them
  *     on one stream or with events.
@@ -360,6 +364,26 @@ pa_status pa_bm_get_stats(const pa_block_manager* bm, pa_bm_stats* out);
 
 /* Reference count of one physical block (-1 for a bad id). */
 int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
+
+/*
+ * Measurement utility, with no counterpart on the pages: the streaming-read
+ * ceiling of this GPU's memory, the roofline of the decode path (which only
+ * reads the cache; a read+write copy benchmark is not its ceiling).
+ * Reads `bytes` bytes at `buf` (device memory, 16-byte aligned, bytes a
+ * multiple of 16) once with every SM and discards them:
+ *   method 0: 128-bit loads that bypass L1, eight in flight per thread,
+ *             every resident thread sweeping the buffer;
+ *   method 1: bulk asynchronous copies (cp.async.bulk, 16 KiB, no multicast)
+ *             into a shared-memory ring per CTA -- the engine the decode
+ *             kernels read their tiles with.
+ * Each CTA XORs a fold of what it read into *sink (device uint64, 8-byte
+ * aligned; its value means nothing, it only keeps the loads alive). A bulk
+ * wait that gives up adds PA_DEV_ERR_TIMEOUT to *dev_error (nullable). Time
+ * it with events on `stream`; buffers larger than L2 measure HBM.
+ * PA_ERR_INVALID_ARG for a bad method, pointer, alignment or size.
+ */
+pa_status pa_read_probe(const void* buf, size_t bytes, int32_t method, uint64_t* sink,
+                        int32_t* dev_error, void* stream);
 
 /* Static description of a status code. */
 const char* pa_status_string(pa_status status);

@@ -57,6 +57,31 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     return LIB
 
 
+# Test-only builds of the same sources with extra defines. "waittest": every
+# K/V tile wait of the decode kernels probes once (PA_TEST_TILE_WAIT_ONCE), so
+# tests can make a bounded wait run out without withholding any copy.
+VARIANTS = {"waittest": ["-DPA_TEST_TILE_WAIT_ONCE"]}
+
+
+def variant_path(name: str) -> str:
+    return os.path.join(PKG, f"libpa_{name}.so")
+
+
+def build_variant(name: str, force: bool = False, verbose: bool = False) -> str:
+    """Compile the test-only library `name` (see VARIANTS) next to libpa.so."""
+    out = variant_path(name)
+    if not force and os.path.exists(out) and \
+            all(os.path.getmtime(f) <= os.path.getmtime(out) for f in _inputs()):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [nvcc()] + NVCC_FLAGS + VARIANTS[name] + ["-I", INCLUDE, "-o", tmp] + sources()
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)

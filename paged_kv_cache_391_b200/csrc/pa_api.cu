@@ -411,4 +411,17 @@ pa_status pa_swap_blocks(void* const* src_k, void* const* src_v, void* const* ds
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
+pa_status pa_read_probe(const void* buf, size_t bytes, int32_t method, uint64_t* sink,
+                        int32_t* dev_error, void* stream) {
+  if (method != 0 && method != 1) return PA_ERR_INVALID_ARG;
+  if (bytes == 0) return PA_OK;
+  if (!buf || !sink || !aligned(buf, 16) || bytes % 16 || !aligned(sink, 8) ||
+      (dev_error && !aligned(dev_error, 4)))
+    return PA_ERR_INVALID_ARG;
+  cudaError_t e = pa::launch_read_probe(buf, bytes, method,
+                                        reinterpret_cast<unsigned long long*>(sink), dev_error,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
 }  // extern "C"

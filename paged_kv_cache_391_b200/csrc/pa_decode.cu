@@ -282,7 +282,7 @@ __device__ __forceinline__ bool attend_item(const ItemArgs<T>& A, uint8_t* smem,
     const int st = (ring + it) % SM::kStages;
     const uint32_t parity = (uint32_t)(((ring + it) / SM::kStages) & 1);
     const int p = pid_of(it);
-    if (!__all_sync(kFull, mbar_wait(&wbars[st], parity))) {
+    if (!__all_sync(kFull, mbar_wait_tile(&wbars[st], parity))) {
       timed_out = true;
       break;
     }
@@ -403,14 +403,17 @@ __device__ __forceinline__ bool attend_item(const ItemArgs<T>& A, uint8_t* smem,
     }
   }
   if (timed_out) {
-    // Let the copies already in flight land (each wait bounded) before the
-    // shared memory is reused or the CTA exits, then report.
+    // Let the copies already in flight (tiles it .. it + kStages - 1) land,
+    // each wait bounded, before the shared memory is reused or the CTA exits,
+    // then report. The ring advances by the phases that completed.
     const int last = min(n_mine, it + SM::kStages);
     for (int k = it; k < last; ++k)
       (void)mbar_wait(&wbars[(ring + k) % SM::kStages], ((ring + k) / SM::kStages) & 1);
     if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
+    ring += (uint32_t)last;
+  } else {
+    ring += (uint32_t)n_mine;
   }
-  ring += (uint32_t)n_mine;
 
   // ---- merge the four warps (log-sum-exp), then write out or the partials
   l_a += __shfl_xor_sync(kFull, l_a, 1);
@@ -985,13 +988,10 @@ static cudaError_t launch_persistent_typed(const DecodeLaunch& a, cudaStream_t s
   auto kern = decode_persistent_kernel<T, D, kTwoRows>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
-  static int per_sm = 0;  // resident CTAs per SM (the same on every device of this arch)
-  if (per_sm == 0) {
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, SM::kAlloc);
-    if (e != cudaSuccess) return e;
-    per_sm = n > 0 ? n : 1;
-  }
+  int per_sm = 0;  // resident CTAs per SM, asked per call (cheap next to the launch)
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, SM::kAlloc);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)

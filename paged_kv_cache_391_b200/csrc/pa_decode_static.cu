@@ -13,12 +13,18 @@
 // Set-up: the first call on a device (with that device current) looks up the
 // array's device address with cudaGetSymbolAddress -- in host code the
 // array's name only stands for it and must never be handed to a kernel. Make
-// that first call before any stream capture on that device.
+// that first call before any stream capture on that device. The address is
+// kept per device together with the id of the CUDA context it belongs to;
+// when the device's context changes (after cudaDeviceReset, the library's
+// device code is loaded again and the array may move) the next call looks
+// the address up again.
 //
 // Sharing: every call on a device uses the same array. Each call writes every
 // partial result it later reads, so nothing has to start at zero, but two
 // calls whose kernels overlap on the GPU (different streams, no ordering
 // between them) race on the array. Order them on one stream, or by events.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "pa.h"
@@ -29,24 +35,60 @@ static __device__ __align__(256) unsigned char g_decode_scratch[PA_STATIC_WORKSP
 namespace {
 
 constexpr int kMaxDevices = 128;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device, looked up once
-// per device.
+struct ScratchSlot {
+  void* addr = nullptr;
+  unsigned long long ctx_id = 0;  // 0: unknown
+};
+
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch[kMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (driver entry
+// points, looked up once); false when there is none or it cannot be read.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
+
+// Device address of g_decode_scratch on the current device, looked up on the
+// first call and again whenever the device's context has changed.
 pa_status scratch_on_current_device(void** addr) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return pa::record_cuda_error(e);
   if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  if (!slot.addr || !have_id || slot.ctx_id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);  // makes the context current if needed
     if (e != cudaSuccess) return pa::record_cuda_error(e);
-    g_scratch_addr[dev] = p;
+    unsigned long long now = 0;
+    slot.addr = p;
+    slot.ctx_id = current_context_id(&now) ? now : 0;
   }
-  *addr = g_scratch_addr[dev];
+  *addr = slot.addr;
   return PA_OK;
 }
 

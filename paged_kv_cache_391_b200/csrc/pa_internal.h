@@ -77,4 +77,8 @@ cudaError_t launch_block_copy(void* const* src_k, void* const* src_v, void* cons
                               int64_t block_bytes, int64_t src_num_blocks,
                               int64_t dst_num_blocks, int32_t* dev_error, cudaStream_t stream);
 
+// Streaming-read probe (pa_read_probe): method 0 = vector loads, 1 = bulk copies.
+cudaError_t launch_read_probe(const void* buf, size_t bytes, int method,
+                              unsigned long long* sink, int32_t* dev_error, cudaStream_t stream);
+
 }  // namespace pa

@@ -28,7 +28,7 @@ EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_bloc
            "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence",
            "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots", "pa_bm_append_slots",
            "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount", "pa_prefill_chunk",
-           "pa_decode_persistent_workspace_size", "pa_decode_persistent")
+           "pa_decode_persistent_workspace_size", "pa_decode_persistent", "pa_read_probe")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             L.pa_decode_static.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                            i32, ctypes.c_float, i32, P, ctypes.c_int, P]
             L.pa_decode_static.restype = ctypes.c_int
+            L.pa_read_probe.argtypes = [P, sz, i32, P, P, P]
+            L.pa_read_probe.restype = ctypes.c_int
             L.pa_copy_blocks.argtypes = [P, P, i32, P, i32, i32, i32, i32, i64, ctypes.c_int, P, P]
             L.pa_copy_blocks.restype = ctypes.c_int
             L.pa_swap_blocks.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i64, i64,
@@ -256,6 +258,17 @@ def decode_static(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                                 _dtype_code(q), _stream(stream, q.device))
     _check(st, "pa_decode_static")
     return out
+
+
+def read_probe(buf: torch.Tensor, sink: torch.Tensor, *, method: int = 0,
+               dev_error: torch.Tensor | None = None, stream=None) -> None:
+    """Stream every byte of `buf` (device, contiguous) through the SMs once:
+    the memory's read ceiling when timed (method 0: vector loads; 1: bulk
+    asynchronous copies into shared memory). `sink`: one device int64."""
+    assert buf.is_contiguous() and sink.dtype == torch.int64 and sink.numel() >= 1
+    st = lib().pa_read_probe(_ptr(buf), buf.numel() * buf.element_size(), int(method),
+                             _ptr(sink), _ptr(dev_error), _stream(stream, buf.device))
+    _check(st, "pa_read_probe")
 
 
 def copy_blocks(k_caches, v_caches, block_mapping: torch.Tensor, *,

@@ -352,36 +352,52 @@ def shared_prefix(seed: int = 394, num_seqs: int = 100, prefix: int = 5000,
                   suffix_lo: int = 16, suffix_hi: int = 512) -> DecodeWorkload:
     """100 sequences whose tables share one 5000-token prefix (313 blocks, the
     last one holding 8 tokens) plus unique suffixes uniform in [16, 512]
-    tokens; H_q = 32, H_kv = 8, D = 128, bf16. This step forks each
-    sequence's copy of the partial prefix block (one copy pair per sequence)
-    and writes every suffix token, the copied block's free slots first; the
-    prefix blocks stay shared and unchanged ("KV Cache Sharing
-    (Copy-on-Write)": 100 users on one 5,000-token system prompt)."""
+    tokens; H_q = 32, H_kv = 8, D = 128, bf16 ("KV Cache Sharing
+    (Copy-on-Write)": 100 users on one 5,000-token system prompt).
+
+    The cache is taken as it stands at a decode step of these sequences: each
+    sequence was forked from the prefix by a copy of the partial prefix block
+    into a block of its own (``notes["fork_pairs"]``, one (src, dst) pair per
+    sequence, as ``copy_blocks`` makes it: the copy's first 8 slots are the
+    shared block's bits), and every suffix token but the last is already
+    cached, the copy's free slots first. The step writes each sequence's
+    newest token and decodes; the 312 full prefix blocks stay shared and
+    unchanged. The fork itself happened before this step, so the step has no
+    copy pairs."""
     rng = np.random.default_rng(seed)
     suf = rng.integers(suffix_lo, suffix_hi, size=num_seqs, endpoint=True)
     n_prefix_blocks = blocks_needed(prefix)
     full = prefix // BLOCK_SIZE
+    tail = prefix % BLOCK_SIZE
     lens = prefix + suf
     need_private = [blocks_needed(int(L)) - full for L in lens]
     nb = int(np.ceil(1.5 * (n_prefix_blocks + sum(need_private))))
     alloc = ToyBlockAllocator(nb, rng)
     shared = alloc.allocate(n_prefix_blocks)
-    tables, pairs, writes = [], [], []
+    tables, forks = [], []
     for s in range(num_seqs):
         private = alloc.allocate(need_private[s])
         tables.append(np.concatenate([shared[:full], private]))
-        if prefix % BLOCK_SIZE:
-            pairs.append([int(shared[full]), int(private[0])])
-        writes += [(s, pos) for pos in range(prefix, int(lens[s]))]
-    # Only the prefix exists before the step; every suffix token is written
-    # by this step, into the private copy's free slots first.
-    fills = [(int(p), BLOCK_SIZE) for p in shared[:full]]
-    if prefix % BLOCK_SIZE:
-        fills.append((int(shared[full]), prefix % BLOCK_SIZE))
-    return _build("shared_prefix", "bf16", 32, 8, 128, 512, seed, rng, tables, fills, lens, nb,
-                  writes, pairs,
-                  {"prefix": prefix, "shared_blocks": full,
-                   "partial_prefix_block": int(shared[full]) if prefix % BLOCK_SIZE else -1})
+        if tail:
+            forks.append([int(shared[full]), int(private[0])])
+    writes = [(s, int(L) - 1) for s, L in enumerate(lens)]
+    # Before the step: the shared prefix, and each sequence's own blocks up to
+    # its newest token (exclusive). A private copy of the partial prefix
+    # block is filled like any block here; its first `tail` slots are then
+    # overwritten with the shared block's bits, as the fork's copy left them.
+    fills = _fills_for([t[full:] for t in tables], np.maximum(lens - 1 - full * BLOCK_SIZE, 0))
+    fills += [(int(p), BLOCK_SIZE) for p in shared[:full]]
+    if tail:
+        fills.append((int(shared[full]), tail))
+    w = _build("shared_prefix", "bf16", 32, 8, 128, 512, seed, rng, tables, fills, lens, nb,
+               writes, [],
+               {"prefix": prefix, "shared_blocks": full,
+                "partial_prefix_block": int(shared[full]) if tail else -1,
+                "fork_pairs": forks})
+    for src, dst in forks:
+        w.k_pool[dst, :, :tail] = w.k_pool[src, :, :tail]
+        w.v_pool[dst, :, :tail] = w.v_pool[src, :, :tail]
+    return w
 
 
 def long_context(seed: int = 395, batch: int = 8, lo: int = 32768, hi: int = 131072,

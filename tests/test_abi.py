@@ -194,3 +194,15 @@ def _prefill(L, **kw):
 ])
 def test_prefill_chunk_rejects_on_the_host(L, kw, status):
     assert _prefill(L, **kw) == status
+
+
+def test_read_probe_rejections(L):
+    """pa_read_probe refuses bad methods, pointers, alignment and sizes on
+    the host, before any launch."""
+    f = L.pa_read_probe
+    assert f(FAKE, 1 << 20, 2, FAKE, None, None) == pa.PA_ERR_INVALID_ARG      # method
+    assert f(None, 1 << 20, 0, FAKE, None, None) == pa.PA_ERR_INVALID_ARG      # buffer
+    assert f(FAKE, 1 << 20, 0, None, None, None) == pa.PA_ERR_INVALID_ARG      # sink
+    assert f(FAKE + 8, 1 << 20, 0, FAKE, None, None) == pa.PA_ERR_INVALID_ARG  # 16-byte base
+    assert f(FAKE, (1 << 20) + 8, 1, FAKE, None, None) == pa.PA_ERR_INVALID_ARG  # 16-byte size
+    assert f(FAKE, 0, 0, None, None, None) == pa.PA_OK                         # nothing to read

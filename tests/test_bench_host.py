@@ -73,3 +73,38 @@ def test_recorded_traffic_follows_the_kernel_sources():
         assert got == (int(nbytes) if h == want else None), key
         assert abs(int(nbytes) / int(alg) - float(ratio)) < 1e-3
     assert set(fam) <= {r[0].partition(":")[0] for r in rows}
+
+
+def _reached(w):
+    used = set()
+    for s, L in enumerate(w.context_lens):
+        used.update(int(b) for b in w.block_tables[s, :W.blocks_needed(int(L))])
+    return used
+
+
+def test_timed_block_copies_never_touch_the_step_cache():
+    """The copies timed on their own: the step's forks when it has any, else
+    copies into blocks that no table reaches (so the timed loop leaves the
+    decode's cache as it was)."""
+    w = W.tiny()
+    pairs, what = bench.timing_copy_pairs(w)
+    assert np.array_equal(pairs, w.copy_pairs) and "step" in what
+    for w in (W.shared_prefix(num_seqs=5, prefix=300, suffix_hi=40), W.mha(batch=4)):
+        pairs, _ = bench.timing_copy_pairs(w)
+        reached = _reached(w)
+        assert len(pairs) == w.num_seqs
+        assert not set(pairs[:, 1].tolist()) & reached
+        assert len(set(pairs[:, 1].tolist())) == len(pairs)
+        assert set(pairs[:, 0].tolist()) <= reached | {w.notes.get("partial_prefix_block", -1)}
+    forks = np.asarray(w.notes.get("fork_pairs", []))
+    assert forks.size == 0   # mha has no forks: the timed copies fork each last block
+
+
+def test_last_block_waste():
+    """Waste = the unused tail of each last block: lengths 16, 17, 31, 1 leave
+    0, 15, 1 and 15 slots of 16, 32, 32 and 16 allocated."""
+    w = W.tiny()
+    w.context_lens = np.array([16, 17, 31, 1], np.int32)
+    r = bench.waste_stats(w)
+    assert r["mean_slots_per_seq"] == 7.75
+    assert r["pct_of_allocated_slots"] == round(100 * 31 / 96, 4)

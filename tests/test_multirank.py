@@ -34,9 +34,10 @@ def _worker(rank, world, port, q):
                             timeout=datetime.timedelta(seconds=60))
     try:
         w = bench.make_workload("gqa", 4, seed_offset=rank)
-        elapsed = 10.0 + 5.0 * rank
-        agg = bench.reduce_over_ranks(elapsed, 20.0 - rank, w.kv_bytes(), w.num_seqs, rank,
-                                      world, device=None)
+        res = {"w": w, "elapsed_ms": 10.0 + 5.0 * rank, "e2e": {"ms": 20.0 - rank},
+               "att_ms": 1.0 + rank, "write_ms": 0.5 - 0.1 * rank, "copy_ms": None,
+               "errors": rank}
+        agg = bench.reduce_over_ranks(res, world, device=None)
         q.put((rank, agg, w.kv_bytes(), int(w.context_lens.sum())))
         dist.barrier()
     finally:
@@ -58,11 +59,17 @@ def test_two_ranks_agree_on_whole_job_figures():
     (r0, a0, kv0, t0), (r1, a1, kv1, t1) = res
     assert a0 == a1                                   # every rank sees the same figures
     assert a0["ms"] == 15.0 and a0["e2e_ms"] == 20.0  # slowest rank
+    assert a0["att_ms"] == 2.0 and a0["write_ms"] == 0.5 and a0["copy_ms"] is None
     assert a0["kv"] == kv0 + kv1 and a0["seqs"] == 8 and a0["errors"] == 1
     assert t0 != t1                                   # ranks ran different (independent) workloads
 
 
 def test_single_rank_is_the_identity():
     import bench
-    agg = bench.reduce_over_ranks(3.0, 4.0, 100, 7, 0, 1)
-    assert agg == {"ms": 3.0, "e2e_ms": 4.0, "kv": 100.0, "seqs": 7.0, "errors": 0}
+    from paged_kv_cache_391_b200 import workloads as W
+    w = W.tiny()
+    res = {"w": w, "elapsed_ms": 3.0, "e2e": None, "att_ms": 2.5, "write_ms": 0.25,
+           "copy_ms": 0.125, "errors": 0}
+    agg = bench.reduce_over_ranks(res, 1)
+    assert agg == {"ms": 3.0, "e2e_ms": 0.0, "att_ms": 2.5, "write_ms": 0.25, "copy_ms": 0.125,
+                   "kv": float(w.kv_bytes()), "seqs": 5.0, "errors": 0}

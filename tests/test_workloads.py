@@ -118,15 +118,29 @@ def test_every_attended_slot_holds_a_token_after_the_step(make):
 
 
 def test_shared_prefix_structure():
+    """The step of the shared-prefix config: the prefix's 312 full blocks are
+    shared, each sequence already owns a copy of the partial prefix block
+    (its first 8 slots are the shared block's bits, as the fork's copy left
+    them) and its suffix up to the newest token; the step writes one token
+    per sequence and copies nothing."""
     w = W.shared_prefix(num_seqs=4, prefix=5000, suffix_hi=40)
     full = 5000 // 16
     assert full == 312 and W.blocks_needed(5000) == 313
     for s in range(1, 4):
         assert np.array_equal(w.block_tables[s, :full], w.block_tables[0, :full])
-    assert len(w.copy_pairs) == 4
-    assert (w.copy_pairs[:, 0] == w.notes["partial_prefix_block"]).all()
-    assert len(set(w.copy_pairs[:, 1].tolist())) == 4
-    assert w.slot_mapping.size == int((w.context_lens - 5000).sum())
+    assert len(w.copy_pairs) == 0
+    forks = np.asarray(w.notes["fork_pairs"])
+    assert forks.shape == (4, 2)
+    assert (forks[:, 0] == w.notes["partial_prefix_block"]).all()
+    assert len(set(forks[:, 1].tolist())) == 4
+    assert (forks[:, 1] == w.block_tables[:, full]).all()
+    src = w.notes["partial_prefix_block"]
+    for dst in forks[:, 1]:
+        assert np.array_equal(w.k_pool[dst, :, :8], w.k_pool[src, :, :8])
+        assert np.array_equal(w.v_pool[dst, :, :8], w.v_pool[src, :, :8])
+    assert w.slot_mapping.size == 4
+    for s in range(4):
+        assert w.slot_mapping[s] == W.slot_of(w.block_tables[s], int(w.context_lens[s]) - 1)
 
 
 def test_config_shapes():

@@ -6,22 +6,24 @@ application that owns all device memory and forbids its plugins from
 allocating, or a decode loop where cudaMalloc/cudaFree (which can synchronise
 the whole device) are not acceptable. pa_decode_static serves them with a
 fixed scratch array compiled into libpa instead of a caller workspace. These
-tests call it through the C ABI and check that it gives what pa_decode gives
-with a caller workspace, on calls made back to back (the scratch keeps the
-previous call's contents), and that sizes beyond the array are refused.
+tests call it through the C ABI and check that, on calls made back to back
+(the scratch keeps the previous call's contents), it gives bit for bit what
+pa_decode gives with a caller workspace -- the same kernels on the same
+inputs -- and the oracle's result within the decode tolerance; and that
+sizes beyond the array are refused before anything is launched.
 
 This file is named so that pytest collects it last.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
+import oracle
 from paged_kv_cache_391_b200 import pa
 from paged_kv_cache_391_b200 import workloads as W
 
-from gpu_helpers import DeviceStep, assert_decode_close, to_f64
+from gpu_helpers import DeviceStep, assert_decode_close, oracle_caches_after_step, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -51,23 +53,26 @@ def test_static_scratch_matches_caller_workspace_on_calls_in_a_row():
         out = torch.full_like(ref, float("nan"))
         assert _static_call(d, out) == pa.PA_OK
         torch.cuda.synchronize()
-        assert_decode_close(to_f64(out), to_f64(ref), "static scratch vs caller workspace")
+        # same kernels, same inputs, same partition size: the same bits
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
         assert int(d.err.item()) == 0
+    # and the result is the oracle's, within the decode tolerance
+    kc, vc = oracle_caches_after_step(a.w)
+    want = oracle.decode(a.w.q, kc, vc, a.w.block_tables, a.w.context_lens, a.w.scale,
+                         a.w.dtype)
+    assert_decode_close(to_f64(out), want, "pa_decode_static vs oracle")
 
 
 def test_sizes_beyond_the_static_scratch_are_refused():
-    w = W.decode_workload("big", [40], num_q_heads=8, num_kv_heads=8, head_dim=128,
-                          dtype="bf16", seed=1)
-    d = DeviceStep(w)
-    # ask for a launch whose partials would not fit: 4096 sequences x 64 heads x 256 partitions
+    # A launch whose partials would not fit: 4096 sequences x 64 heads x 256
+    # partitions. No buffer is passed at all, so even a check order that
+    # regressed could not launch anything (it would return
+    # PA_ERR_INVALID_ARG instead of the size status asserted here).
     need = pa.decode_workspace_size(4096, 64, 128, 131072, 512)
     assert need > pa.PA_STATIC_WORKSPACE_BYTES
-    out = torch.full_like(d.out, 7.0)
     st = pa.lib().pa_decode_static(
-        out.data_ptr(), d.q.data_ptr(), d.k_cache.data_ptr(), d.v_cache.data_ptr(),
-        d.bt.data_ptr(), d.bt.shape[1], d.cl.data_ptr(), 4096, 64, 8, 128, 16, w.num_blocks,
-        131072, ctypes.c_float(w.scale), 512, None, pa.PA_DTYPE_BF16,
+        None, None, None, None, None, 8192, None, 4096, 64, 8, 128, 16, 1 << 20,
+        131072, ctypes.c_float(0.088), 512, None, pa.PA_DTYPE_BF16,
         torch.cuda.current_stream().cuda_stream)
     assert st == pa.PA_ERR_WORKSPACE_TOO_SMALL
     torch.cuda.synchronize()
-    assert (out == 7.0).all()   # nothing was launched
