@@ -191,23 +191,40 @@ pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
  * Frontier: Speculative Decoding and Beyond"). With one token per sequence it
  * equals pa_decode bit for bit.
  * Two implementations, chosen per call: when max_query_len * group_size >= 64,
- * head_dim is 128, group_size is a power of two and partition_tokens is 0 or a
- * multiple of 64, the chunk runs on the tcgen05 tensor cores (accumulators in
- * tensor memory, one CTA per pair of 128-row query tiles); otherwise on the
- * 16-row mma.sync tiles of pa_decode. Both are within the same tolerance of
- * the exact result; they are not bitwise equal to each other.
+ * head_dim is 128, group_size is a power of two and the context is not split
+ * or partition_tokens is a multiple of 128, the chunk runs on the tcgen05
+ * tensor cores (accumulators in tensor memory, one CTA per pair of 128-row
+ * query tiles, 128 keys per step); otherwise on the 16-row mma.sync tiles of
+ * pa_decode. Both are within the same tolerance of the exact result; they are
+ * not bitwise equal to each other.
  *   out, q          device, [num_q_tokens][num_q_heads][head_dim]
  *   q_start         device int32 [num_seqs + 1], non-decreasing, q_start[0] = 0
  *   max_query_len   host upper bound of Tq (sizes the launch); Tq must also be
  *                   <= context_lens[s]
  *   workspace       >= pa_decode_workspace_size(num_q_tokens, num_q_heads,
- *                   head_dim, max_context_len, partition_tokens) bytes
+ *                   head_dim, max_context_len, partition_tokens) bytes (the
+ *                   split partials; NULL when that is 0). On the tcgen05 path,
+ *                   with >= pa_prefill_chunk_workspace_size(...) bytes
+ *                   (256-byte aligned), a plan kernel first lists the work
+ *                   items by descending key count in the space after the
+ *                   partials and the chunk kernel takes them in that order
+ *                   (longest first; fewer idle SMs in the last wave); with
+ *                   less it runs in grid order. Same result either way.
  *   other arguments as for pa_decode. A sequence whose query range falls
  *   outside [0, num_q_tokens) is skipped, one whose Tq exceeds max_query_len
  *   or its context length is clamped; both are counted in dev_error. With a
  *   malformed q_start the output rows of the sequences involved are undefined
  *   (never written out of bounds).
  */
+/* Workspace bytes for pa_prefill_chunk's longest-first order: the split
+ * partials (pa_decode_workspace_size of num_q_tokens rows) plus, when the call
+ * takes the tcgen05 path, 8 bytes per possible (sequence, query-tile pair,
+ * partition) item and 256 bytes. 0 if no workspace is needed. */
+size_t pa_prefill_chunk_workspace_size(int32_t num_q_tokens, int32_t num_seqs,
+                                       int32_t num_q_heads, int32_t group_size, int32_t head_dim,
+                                       int32_t max_query_len, int32_t max_context_len,
+                                       int32_t partition_tokens);
+
 pa_status pa_prefill_chunk(void* out, const void* q, const int32_t* q_start,
                            int32_t num_q_tokens, int32_t max_query_len, const void* k_cache,
                            const void* v_cache, const int32_t* block_tables,

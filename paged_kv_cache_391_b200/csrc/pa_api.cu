@@ -178,6 +178,29 @@ size_t pa_decode_persistent_workspace_size(int32_t num_seqs, int32_t num_q_heads
          round256((size_t)num_seqs * parts * sizeof(uint32_t)) + 256;
 }
 
+// The chunk path's plan (longest-first order of the tcgen05 kernel's work):
+// item list and counter after the partials, or 0 when the tcgen05 path does
+// not apply.
+size_t chunk_plan_bytes(int32_t num_seqs, int32_t group_size, int32_t head_dim,
+                        int32_t max_query_len, int64_t parts, int32_t partition_tokens) {
+  if (num_seqs <= 0 || group_size <= 0 ||
+      !pa::prefill_tc_eligible(head_dim, group_size, max_query_len, parts, partition_tokens))
+    return 0;
+  const int64_t items = pa::prefill_tc_max_items(num_seqs, max_query_len, group_size, parts);
+  return round256((size_t)items * 8) + 256;
+}
+
+size_t pa_prefill_chunk_workspace_size(int32_t num_q_tokens, int32_t num_seqs,
+                                       int32_t num_q_heads, int32_t group_size, int32_t head_dim,
+                                       int32_t max_query_len, int32_t max_context_len,
+                                       int32_t partition_tokens) {
+  if (num_q_tokens <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  return pa_decode_workspace_size(num_q_tokens, num_q_heads, head_dim, max_context_len,
+                                  partition_tokens) +
+         chunk_plan_bytes(num_seqs, group_size, head_dim, max_query_len,
+                          max_partitions(max_context_len, partition_tokens), partition_tokens);
+}
+
 }  // extern "C"
 
 namespace {
@@ -268,6 +291,8 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   a.bf16 = dtype == PA_DTYPE_BF16;
   a.items = nullptr;
   a.plan = nullptr;
+  a.chunk_items = nullptr;
+  a.chunk_plan = nullptr;
   if (persistent) {
     char* tail = static_cast<char*>(workspace) + need;
     a.items = reinterpret_cast<uint32_t*>(tail);
@@ -278,6 +303,18 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   // Long query chunks (at least 64 rows of (token, head) per KV head) are a
   // dense contraction: run them on the tcgen05 tensor cores.
   if (q_start && (int64_t)max_query_len * group_size >= 64 && pa::prefill_tc_supported(a)) {
+    // With room after the partials (pa_prefill_chunk_workspace_size), a plan
+    // kernel orders the work longest first; otherwise the grid's order.
+    const size_t plan = chunk_plan_bytes(num_seqs, group_size, head_dim, max_query_len, parts,
+                                         partition_tokens);
+    if (plan && workspace && aligned(workspace, 256) && workspace_bytes >= need + plan &&
+        pa::prefill_tc_max_items(num_seqs, max_query_len, group_size, parts) * num_kv_heads <=
+            0x7fffffff) {
+      char* tail = static_cast<char*>(workspace) + need;
+      const int64_t items = pa::prefill_tc_max_items(num_seqs, max_query_len, group_size, parts);
+      a.chunk_items = reinterpret_cast<uint2*>(tail);
+      a.chunk_plan = reinterpret_cast<int32_t*>(tail + round256((size_t)items * 8));
+    }
     CUtensorMap tm_q;
     st = encode_query_map(&tm_q, q, num_q_tokens, num_q_heads, head_dim, group_size, dtype);
     if (st != PA_OK) return st;

@@ -76,17 +76,6 @@ __device__ __forceinline__ uint32_t tile_off(int t, int d) {
   return (uint32_t)((d >> 6) * 2048 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4) + (d & 7) * 2);
 }
 
-// Programmatic dependent launch: a kernel launched with the attribute may
-// start while the previous kernel in the stream finishes; it reads no global
-// memory before griddep_wait(), which returns once that kernel has completed
-// and its writes are visible. Without the attribute both are no-ops.
-__device__ __forceinline__ void griddep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // The arguments every work item shares.
 template <typename T>
 struct ItemArgs {

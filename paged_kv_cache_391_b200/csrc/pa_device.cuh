@@ -102,6 +102,17 @@ __device__ __forceinline__ bool mbar_wait_tile(uint64_t* bar, uint32_t parity) {
 #endif
 }
 
+// Programmatic dependent launch: a kernel launched with the attribute may
+// start while the previous kernel in the stream finishes; it reads no global
+// memory before griddep_wait(), which returns once that kernel has completed
+// and its writes are visible. Without the attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 // Tiled 4-D tensor load into this CTA's shared memory, completion counted on
 // `bar` in bytes. No multicast.

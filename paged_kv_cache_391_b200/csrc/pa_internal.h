@@ -40,6 +40,10 @@ struct DecodeLaunch {
   int bf16;          // 0 = fp16, 1 = bf16
   uint32_t* items;   // work queue: [num_seqs * max_parts] (seq << 16) | part
   int32_t* plan;     // [0] = items listed, [1] = work counter
+  // tcgen05 chunk path, longest first (NULL: grid order): [max items] of
+  // {sequence, pair * max_parts + partition}, then [0] = items listed
+  uint2* chunk_items;
+  int32_t* chunk_plan;
 };
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
@@ -56,6 +60,12 @@ cudaError_t launch_reduce(const DecodeLaunch& a, cudaStream_t stream);
 // (partition kernel; the caller runs launch_reduce after it). tm_q maps q as
 // [tokens][H_q][D] with boxes of 64 columns x group heads x 128/group tokens.
 bool prefill_tc_supported(const DecodeLaunch& a);
+// Whether a chunk call takes the tcgen05 path (the same test pa_prefill_chunk
+// applies), and the most (sequence, tile pair, partition) items it can have.
+bool prefill_tc_eligible(int32_t head_dim, int32_t group, int32_t max_query_len, int64_t parts,
+                         int32_t partition_tokens);
+int64_t prefill_tc_max_items(int32_t num_seqs, int32_t max_query_len, int32_t group,
+                             int64_t parts);
 cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q, cudaStream_t stream);
 
 // Records a CUDA error for pa_last_cuda_error() and returns PA_ERR_CUDA.

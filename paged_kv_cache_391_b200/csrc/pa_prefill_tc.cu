@@ -10,23 +10,28 @@
 //
 // One CTA per (pair of 128-row query tiles, partition, KV head, sequence);
 // tile rows are (query token, head) pairs of the KV head's query group. Both
-// tiles share every K/V tile the CTA loads, and while one tile's softmax runs
-// the tensor core works on the other's (the two-tile ping-pong of
-// FlashAttention-4). 320 threads, one CTA per SM:
+// tiles share every K/V tile the CTA loads. 320 threads, one CTA per SM:
 //  * warps 0-3 and 4-7: softmax of tile 0 and tile 1. Thread r of a
 //    warpgroup owns row r of its tile: TMEM lane r of its S, P and O.
-//  * warp 8: TMA loads (Q once; per step K and V of 4 cache blocks = 64 keys,
-//    each in its own 3-stage ring, eight lanes issuing a ring's eight boxes).
-//  * warp 9, one lane: every MMA, for tiles i = 0, 1:
-//      S_i[j%2] = Q_i K_j^T   (M=128, N=64, K=D; Q and K K-major in shared memory)
-//      O_i     += P_i,j V_j   (M=128, N=D, K=64; P K-major, V MN-major)
-//    S is double-buffered in TMEM so S(j+1) runs while the softmax of step j
-//    does; each softmax writes P_i,j (bf16, 128-byte swizzled) into its
-//    tile's shared buffer once P.V(j-1) has read P_i,j-1. A K (V) stage is
-//    refilled once the S (P.V) MMAs that read it committed its "empty"
-//    barrier. Loads and MMAs sit in separate warps on separate schedulers,
-//    so neither waits on the other's instruction issue.
-//    TMEM: tile i at columns 256 i: S0 [0,64), S1 [64,128), O [128,256).
+//  * warp 8: TMA loads (Q once; per step K and V of 8 cache blocks = 128
+//    keys, each in its own 2-stage ring, sixteen lanes issuing a ring's
+//    sixteen boxes).
+//  * warp 9, one lane: every MMA:
+//      S_i(j)  = Q_i K_j^T      (M=128, N=128 keys, K=D; Q, K K-major in smem)
+//      O_i    += P_i(j) V_j     (M=128, N=D, K=128 keys; P in TMEM, V MN-major
+//                                in smem)
+//    P_i(j) (bf16) is written by the softmax over the first 64 columns of
+//    S_i(j), so the tensor core reads only V from shared memory for P.V and
+//    Q, K for S: per 128 keys 8 KiB of operands per 64-cycle MMA at most.
+//    Issue order S_0(j), P.V_1(j-1), S_1(j), P.V_0(j), S_0(j+1), ...: each
+//    tile's softmax has the time of two MMA groups (the other tile's) to
+//    finish, the two softmaxes alternate instead of competing, and S_i(j+1)
+//    is issued after P.V_i(j), which has read P_i(j) from the same columns
+//    (tcgen05 MMAs of one thread run in issue order). The commit that
+//    signals S_i(j) also covers P.V_i(j-1), so the softmax may rescale O_i
+//    as soon as it sees S_i(j).
+//    TMEM: tile i at columns 256 i: S (P over its first half) [0,128),
+//    O [128,256).
 // Online softmax per row in fp32, base 2 (hardware ex2); a row's reference
 // maximum and O are only rescaled when the maximum grows by more than 2^8.
 // Keys past the context, past the row's causal limit, or in a block with a bad
@@ -47,31 +52,29 @@ namespace {
 
 constexpr int kRows = 128;                 // query rows per tile (M)
 constexpr int kTiles = 2;                  // query tiles per CTA
-constexpr int kKeys = 64;                  // keys per step (4 cache blocks)
+constexpr int kKeys = 128;                 // keys per step (8 cache blocks)
 constexpr int kStepBlocks = kKeys / 16;
 constexpr int kD = 128;                    // head dim of this path
 constexpr int kChunks = kD / 64;           // 128-byte swizzle columns of a row
-constexpr int kStages = 3;                 // K and V ring depth
+constexpr int kStages = 2;                 // K and V ring depth
 constexpr int kSoftmaxWarps = 4 * kTiles;
 constexpr int kLoadWarp = kSoftmaxWarps;       // TMA loads
 constexpr int kMmaWarp = kSoftmaxWarps + 1;    // tcgen05.mma issue
 constexpr int kThreadsTc = (kSoftmaxWarps + 2) * 32;
-constexpr uint32_t kTileCols = 256;        // per tile: S0 [0,64) S1 [64,128) O [128,256)
+constexpr uint32_t kTileCols = 256;        // per tile: S / P [0,128), O [128,256)
 constexpr uint32_t kTmemCols = kTiles * kTileCols;
 constexpr uint32_t kOCol = 128;
 
 constexpr int kQBytes = kRows * kD * 2;            // 32 KiB per tile: [chunk][128 rows][128 B]
-constexpr int kKBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]
-constexpr int kVBytes = kKeys * kD * 2;            // 16 KiB: [chunk][64 keys][128 B]
-constexpr int kPBytes = kRows * kKeys * 2;        // 16 KiB per tile: [128 rows][128 B] bf16 P
+constexpr int kKBytes = kKeys * kD * 2;            // 32 KiB: [chunk][128 keys][128 B]
+constexpr int kVBytes = kKeys * kD * 2;            // 32 KiB: [chunk][128 keys][128 B]
 constexpr int kQOff = 0;                           // Q tiles 0, 1
 constexpr int kKOff = kTiles * kQBytes;            // K stages
 constexpr int kVOff = kKOff + kStages * kKBytes;   // V stages
-constexpr int kPOff = kVOff + kStages * kVBytes;   // P tiles 0, 1
-constexpr int kBarOff = kPOff + kTiles * kPBytes;
-// barriers: q_full, k_full[3], k_empty[3], v_full[3], v_empty[3],
-// s_full[2 tiles][2], p_ready[2], pv_done[2]; then the TMEM address
-constexpr int kNumBars = 1 + 4 * kStages + 4 * kTiles;
+constexpr int kBarOff = kVOff + kStages * kVBytes;
+// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2],
+// s_full[2 tiles], p_ready[2 tiles], o_done, mma_drain; then the TMEM address
+constexpr int kNumBars = 1 + 4 * kStages + 2 * kTiles + 2;
 constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kTmemSlotOff + 16;
 // The dynamic shared memory is declared 1024-byte aligned and the kernel
@@ -85,6 +88,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// 2^x on the FMA and integer pipes, for a share of the exponentials so that
+// the MUFU pipe (16 results per clock per SM, as few as the tensor core needs
+// at D = 128) is not the limit: x = n + f with n = round(x) (by adding
+// 1.5 * 2^23, which leaves n in the low mantissa bits) and f in [-0.5, 0.5];
+// 2^f by a cubic fitted here to minimise the relative error on that interval
+// (iteratively reweighted least squares over Chebyshev nodes: max relative
+// error 7.5e-5, below bf16's 2^-9 rounding of P); n is added to the exponent
+// field. Inputs below -126 give 0 (as ex2.approx.ftz does there).
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;          // 1.5 * 2^23: round x to an integer
+  const float f = x - (t - 12582912.f);    // in [-0.5, 0.5]
+  float p = fmaf(0.05517144f, f, 0.24261114f);
+  p = fmaf(p, f, 0.69326103f);
+  p = fmaf(p, f, 0.99992806f);
+  const int n = __float_as_int(t) - 0x4B400000;  // round(x), from the low mantissa bits
+  const float y = __int_as_float(__float_as_int(p) + (n << 23));
+  return x > -126.f ? y : 0.f;
+}
+
+// Every kPolyEvery-th pair of exponentials of a row is taken by poly_exp2
+// (0: none).
+#ifndef PA_TC_POLY_EVERY
+#define PA_TC_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = PA_TC_POLY_EVERY;
 
 // A row's running maximum is only moved (and O rescaled) when the new
 // maximum exceeds it by more than 2^8: until then P is taken against the
@@ -102,7 +132,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                       const int32_t* __restrict__ block_tables, int bt_stride,
                       const int32_t* __restrict__ context_lens, int num_q_heads, int group,
                       int64_t num_blocks, int max_context_len, float scale_log2,
-                      int part_blocks, int max_parts, int32_t* __restrict__ dev_error) {
+                      int part_blocks, int max_parts, int32_t* __restrict__ dev_error,
+                      const uint2* __restrict__ items, const int32_t* __restrict__ plan,
+                      int num_kv_heads) {
   using E = Elem<T>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
@@ -112,9 +144,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint64_t* k_empty = k_full + kStages;             // [stage]
   uint64_t* v_full = k_empty + kStages;             // [stage]
   uint64_t* v_empty = v_full + kStages;             // [stage]
-  uint64_t* s_full = v_empty + kStages;             // [tile * 2 + buffer]
-  uint64_t* p_ready = s_full + 2 * kTiles;          // [tile]
-  uint64_t* pv_done = p_ready + kTiles;             // [tile]
+  uint64_t* s_full = v_empty + kStages;             // [tile]
+  uint64_t* p_ready = s_full + kTiles;              // [tile]
+  uint64_t* o_done = p_ready + kTiles;
+  uint64_t* mma_drain = o_done + 1;                 // failure path only
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlotOff);
 
   if (smem_addr(smem) & 1023) {  // the 128-byte swizzle needs 1024-byte aligned tiles
@@ -122,9 +155,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       atomicAdd(dev_error, 1);
     return;
   }
-  const int kvh = blockIdx.y, seq = blockIdx.z;
-  const int part = (int)(blockIdx.x % (unsigned)max_parts);
-  const int qtile = (int)(blockIdx.x / (unsigned)max_parts) * kTiles;  // the CTA's first tile
+  // The CTA's work: (pair of query tiles, partition, KV head, sequence) from
+  // the grid, or -- longest first -- from the plan (a 1-D grid; item w / H_kv
+  // of the plan's list, KV head w % H_kv).
+  int kvh, seq, part, qtile;
+  if (plan) {
+    griddep_wait();  // the plan kernel's list is complete and visible
+    const int64_t w = blockIdx.x;
+    if (w >= (int64_t)plan[0] * num_kv_heads) return;
+    const uint2 it = items[w / num_kv_heads];
+    kvh = (int)(w % num_kv_heads);
+    seq = (int)it.x;
+    part = (int)(it.y % (unsigned)max_parts);
+    qtile = (int)(it.y / (unsigned)max_parts) * kTiles;
+  } else {
+    kvh = blockIdx.y;
+    seq = blockIdx.z;
+    part = (int)(blockIdx.x % (unsigned)max_parts);
+    qtile = (int)(blockIdx.x / (unsigned)max_parts) * kTiles;  // the CTA's first tile
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool counter = part == 0 && kvh == 0 && qtile == 0 && tid == 0 && dev_error;
 
@@ -152,7 +201,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   if (part >= n_parts) return;
   const int key_begin = part * part_blocks * 16;
   const int t_last = min(t0 + kTiles * tok_per_tile, Tq) - 1;  // last query token of the CTA
-  // keys this tile can see in this partition: up to the last row's causal limit
+  // keys this CTA can see in this partition: up to the last row's causal limit
   const int key_end = min(min((part + 1) * part_blocks * 16, L), L - Tq + t_last + 1);
   const int n_steps = key_end > key_begin ? (key_end - key_begin + kKeys - 1) / kKeys : 0;
   const int q_head0 = kvh * group;
@@ -167,11 +216,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < kTiles; ++i) {
-      mbar_init(&s_full[2 * i], 1);
-      mbar_init(&s_full[2 * i + 1], 1);
+      mbar_init(&s_full[i], 1);
       mbar_init(&p_ready[i], 4 * 32);
-      mbar_init(&pv_done[i], 1);
     }
+    mbar_init(o_done, 1);
+    mbar_init(mma_drain, 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -187,15 +236,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t q_s = smem_addr(smem + kQOff);
   auto stage_k = [&](int st) { return smem + kKOff + st * kKBytes; };
   auto stage_v = [&](int st) { return smem + kVOff + st * kVBytes; };
-  uint8_t* p_buf = smem + kPOff;
   const int32_t* bt_row = block_tables + (size_t)seq * bt_stride;
 
   if (warp == kLoadWarp) {
     // ============================ TMA loads =================================
     // The whole warp runs the control flow, so the block table is read 32
     // entries per coalesced load and broadcast by shuffle. Per step and ring
-    // (K, then V) lane 0 posts the expected bytes and lanes 0-7 issue the
-    // step's eight box copies (4 cache blocks x 2 column chunks) in one
+    // (K, then V) lane 0 posts the expected bytes and lanes 0-15 issue the
+    // step's sixteen box copies (8 cache blocks x 2 column chunks) in one
     // instruction. A stage is refilled once the MMAs that read it committed
     // its "empty" barrier; the loads run up to kStages steps ahead.
     const int lb_first = key_begin / 16;
@@ -219,19 +267,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const int v = w == win ? pid_cur : pid_nxt;
       return __shfl_sync(0xffffffffu, v, i & 31);
     };
-    // K (or V) of step j's four cache blocks into stage j % kStages; blocks
+    // K (or V) of step j's eight cache blocks into stage j % kStages; blocks
     // past the keys or with a bad table entry are not loaded.
     auto load = [&](int j, bool is_v) {
       const int st = j % kStages;
       uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
       uint8_t* dst = is_v ? stage_v(st) : stage_k(st);
       const CUtensorMap* map = is_v ? &tm_v : &tm_k;
-      while (((j * kStepBlocks) >> 5) > win) {  // a step's 4 entries share one window
+      while (((j * kStepBlocks) >> 5) > win) {  // a step's 8 entries share one window
         ++win;
         pid_cur = pid_nxt;
         pid_nxt = load_window(win + 1);
       }
-      const int b = (lane >> 1) & (kStepBlocks - 1), c = lane & 1;  // lanes 0-7: block, chunk
+      const int b = (lane >> 1) & (kStepBlocks - 1), c = lane & 1;  // lanes 0-15: block, chunk
       const int pid = pid_of(j * kStepBlocks + b);
       const bool mine = lane < kStepBlocks * kChunks && pid >= 0;
       const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, mine)) * 2048u;
@@ -282,76 +330,82 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp == kMmaWarp) {
     // ============================== MMAs ====================================
-    // One lane issues every tcgen05.mma, in the order S(j) of both tiles,
-    // then P.V(j-1) of both tiles, so S(j) runs while the softmax of step
-    // j-1 finishes. Descriptors are built once and offset per MMA.
+    // One lane issues every tcgen05.mma in the order S_0(j), P.V_1(j-1),
+    // S_1(j), P.V_0(j). Descriptors are built once and offset per MMA.
     const bool leader = lane == 0;
     const uint32_t id_s = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kKeys, false, false);
     const uint32_t id_pv = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kD, false, true);
     const uint64_t dq = tc::smem_desc_sw128(q_s, 16, 1024);
     const uint64_t dk = tc::smem_desc_sw128(smem_addr(stage_k(0)), 16, 1024);
     const uint64_t dv = tc::smem_desc_sw128(smem_addr(stage_v(0)), kKeys * 128, 1024);
-    const uint64_t dp = tc::smem_desc_sw128(smem_addr(p_buf), 16, 1024);
-    uint64_t* last_bar = nullptr;  // barrier of the last commit, and its parity
-    uint32_t last_parity = 0;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity));
     };
-    if (n_steps > 0 && !wait_all(q_full, 0)) failed = true;
-    for (int j = 0; j <= n_steps && !failed; ++j) {
-      if (j < n_steps) {
-        // S(j): its TMEM buffer j % 2 was read by softmax(j-2), whose p_ready
-        // was awaited before P.V(j-2).
-        const int st = j % kStages, buf = j & 1;
-        if (!wait_all(&k_full[st], (uint32_t)((j / kStages) & 1))) { failed = true; break; }
-        tc::fence_after_sync();
-        if (leader) {
-          const uint64_t dks = dk + (uint64_t)((st * kKBytes) >> 4);
+    // S_i(j) = Q_i K_j^T into tile i's S columns; commit to s_full[i]
+    auto issue_s = [&](int i, int j) {
+      const uint64_t dks = dk + (uint64_t)(((j % kStages) * kKBytes) >> 4);
+      if (leader) {
 #pragma unroll
-          for (int i = 0; i < kTiles; ++i) {
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (kk & 3) * 32;  // 16 columns = 32 bytes into the row
-              const uint64_t a = dq + (uint64_t)((i * kQBytes + (kk >> 2) * (kRows * 128) + off) >> 4);
-              const uint64_t b = dks + (uint64_t)(((kk >> 2) * (kKeys * 128) + off) >> 4);
-              tc::mma_f16(tmem + (uint32_t)(i * kTileCols + buf * kKeys), a, b, id_s, kk > 0);
-            }
-            tc::commit(&s_full[2 * i + buf]);
-          }
-          tc::commit(&k_empty[st]);  // K stage st free once these MMAs completed
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;  // 16 columns = 32 bytes into the row
+          const uint64_t a = dq + (uint64_t)((i * kQBytes + (kk >> 2) * (kRows * 128) + off) >> 4);
+          const uint64_t b = dks + (uint64_t)(((kk >> 2) * (kKeys * 128) + off) >> 4);
+          tc::mma_f16(tmem + (uint32_t)(i * kTileCols), a, b, id_s, kk > 0);
         }
-        last_bar = &k_empty[st];
-        last_parity = (uint32_t)((j / kStages) & 1);
+        tc::commit(&s_full[i]);
       }
-      if (j >= 1) {
-        // P.V(j-1) of both tiles, once V(j-1) landed and each tile's P is in place
-        const int jp = j - 1, st = jp % kStages;
-        if (!wait_all(&v_full[st], (uint32_t)((jp / kStages) & 1))) { failed = true; break; }
-        const uint64_t dvs = dv + (uint64_t)((st * kVBytes) >> 4);
-        for (int i = 0; i < kTiles; ++i) {
-          if (!wait_all(&p_ready[i], (uint32_t)(jp & 1))) { failed = true; break; }
-          tc::fence_after_sync();
-          if (leader) {
+    };
+    // O_i += P_i(j) V_j, P from TMEM (the first 64 columns of tile i's S)
+    auto issue_pv = [&](int i, int j) {
+      const uint64_t dvs = dv + (uint64_t)(((j % kStages) * kVBytes) >> 4);
+      if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk) {
-              const uint64_t a = dp + (uint64_t)((i * kPBytes + kk * 32) >> 4);
-              const uint64_t b = dvs + (uint64_t)((kk * 2048) >> 4);
-              tc::mma_f16(tmem + (uint32_t)(i * kTileCols) + kOCol, a, b, id_pv, jp > 0 || kk > 0);
-            }
-            tc::commit(&pv_done[i]);
-          }
-          last_bar = &pv_done[i];
-          last_parity = (uint32_t)(jp & 1);
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint64_t b = dvs + (uint64_t)((kk * 2048) >> 4);
+          tc::mma_f16_tmem_a(tmem + (uint32_t)(i * kTileCols) + kOCol,
+                             tmem + (uint32_t)(i * kTileCols) + (uint32_t)(kk * 8), b, id_pv,
+                             j > 0 || kk > 0);
         }
-        if (failed) break;
-        if (leader) tc::commit(&v_empty[st]);
-        last_bar = &v_empty[st];
-        last_parity = (uint32_t)((jp / kStages) & 1);
+      }
+    };
+    if (n_steps > 0 && !wait_all(q_full, 0)) failed = true;
+    for (int j = 0; j < n_steps && !failed; ++j) {
+      const int st = j % kStages;
+      if (!wait_all(&k_full[st], (uint32_t)((j / kStages) & 1))) { failed = true; break; }
+      tc::fence_after_sync();
+      issue_s(0, j);
+      if (j > 0) {  // P.V_1(j-1): V(j-1) landed (awaited before P.V_0(j-1))
+        if (!wait_all(&p_ready[1], (uint32_t)((j - 1) & 1))) { failed = true; break; }
+        tc::fence_after_sync();
+        issue_pv(1, j - 1);
+        if (leader) tc::commit(&v_empty[(j - 1) % kStages]);
+      }
+      issue_s(1, j);
+      if (leader) tc::commit(&k_empty[st]);  // K stage st free once S_0(j), S_1(j) completed
+      if (!wait_all(&v_full[st], (uint32_t)((j / kStages) & 1))) { failed = true; break; }
+      if (!wait_all(&p_ready[0], (uint32_t)(j & 1))) { failed = true; break; }
+      tc::fence_after_sync();
+      issue_pv(0, j);
+    }
+    if (!failed && n_steps > 0) {
+      const int jl = n_steps - 1;
+      if (!wait_all(&p_ready[1], (uint32_t)(jl & 1))) {
+        failed = true;
+      } else {
+        tc::fence_after_sync();
+        issue_pv(1, jl);
+        if (leader) {
+          tc::commit(&v_empty[jl % kStages]);
+          tc::commit(o_done);  // both tiles' O are final once this completes
+        }
       }
     }
     if (failed) {
-      // The MMAs already issued finish (bounded wait) before TMEM is released.
-      if (last_bar) (void)mbar_wait(last_bar, last_parity);
+      // The MMAs already issued finish (bounded wait) before TMEM is released:
+      // a commit covers every MMA this thread issued before it. o_done stays
+      // unsignalled, so the softmax warps time out instead of reading O.
+      if (leader) tc::commit(mma_drain);
+      (void)mbar_wait(mma_drain, 0);
       if (leader && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
     }
   } else {
@@ -367,9 +421,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     float m = -INFINITY, l = 0.f;                        // reference maximum (log2 units)
     // keys every row of the tile may see: up to the first row's causal limit
     const int key_all = min(key_end, L - Tq + tt0 + 1);
-    uint64_t* my_s_full = &s_full[2 * tile];
-    uint64_t* my_pv_done = &pv_done[tile];
-    uint8_t* my_p = p_buf + tile * kPBytes;
     // Validity of the table entries of a step (a bit per cache block), loaded
     // one step ahead so the table reads never wait in the loop.
     auto bad_blocks = [&](int j) {
@@ -387,24 +438,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     };
     int bad_next = n_steps > 0 ? bad_blocks(0) : 0;
     for (int j = 0; j < n_steps; ++j) {
-      const int buf = j & 1, st = j % kStages;
+      const int st = j % kStages;
       const int kb = key_begin + j * kKeys;
       const int bad_mask = bad_next;
       if (j + 1 < n_steps) bad_next = bad_blocks(j + 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&my_s_full[buf], (j >> 1) & 1))) { failed = true; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], (uint32_t)(j & 1)))) { failed = true; break; }
       tc::fence_after_sync();
-      float s[64];
-      {
-        float a[32], b2[32];
-        tc::tmem_ld32(lane_addr + (uint32_t)(buf * kKeys), a);
-        tc::tmem_ld32(lane_addr + (uint32_t)(buf * kKeys + 32), b2);
-        tc::tmem_wait_ld();
+      float s[kKeys];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = a[i];
-          s[32 + i] = b2[i];
-        }
+      for (int c = 0; c < kKeys / 32; ++c) {
+        float v[32];
+        tc::tmem_ld32(lane_addr + (uint32_t)(c * 32), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[32 * c + i] = v[i];
       }
+      tc::tmem_wait_ld();
       // Logits in log2 units are s * scale_log2. Steps wholly inside the
       // tile's causal horizon need no mask (scale folded into the exp's FMA);
       // otherwise scale first and give masked keys -inf.
@@ -413,7 +461,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (need_mask) {
         mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < kKeys; ++i) {
           const int kp = kb + i;
           const bool ok = kp < key_end && kp <= lim && !((bad_mask >> (i >> 4)) & 1);
           s[i] = ok ? s[i] * scale_log2 : -INFINITY;
@@ -421,13 +469,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         cc = 1.f;
       } else {
-        float hi = s[0], lo = s[0];
+        float hi0 = s[0], lo0 = s[0], hi1 = s[1], lo1 = s[1];
 #pragma unroll
-        for (int i = 1; i < 64; ++i) {
-          hi = fmaxf(hi, s[i]);
-          lo = fminf(lo, s[i]);
+        for (int i = 2; i < kKeys; i += 2) {
+          hi0 = fmaxf(hi0, s[i]);
+          lo0 = fminf(lo0, s[i]);
+          hi1 = fmaxf(hi1, s[i + 1]);
+          lo1 = fminf(lo1, s[i + 1]);
         }
-        mx = (scale_log2 >= 0.f ? hi : lo) * scale_log2;
+        mx = (scale_log2 >= 0.f ? fmaxf(hi0, hi1) : fminf(lo0, lo1)) * scale_log2;
         cc = scale_log2;
       }
       float alpha = 1.f;
@@ -437,25 +487,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         m = m_new;
       }
       const float m_use = m == -INFINITY ? 0.f : m;
-      uint32_t pk[32];
-      float psum = 0.f;
+      // P_j row r: 128 bf16 = 64 columns over the S columns already read
+      float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = fast_exp2(fmaf(s[2 * i], cc, -m_use));
-        const float p1 = fast_exp2(fmaf(s[2 * i + 1], cc, -m_use));
-        psum += p0 + p1;
-        pk[i] = E::pack(p0, p1);
+      for (int c = 0; c < kKeys / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const bool poly = kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == 0;
+          const float x0 = fmaf(s[32 * c + 2 * i], cc, -m_use);
+          const float x1 = fmaf(s[32 * c + 2 * i + 1], cc, -m_use);
+          const float p0 = poly ? poly_exp2(x0) : fast_exp2(x0);
+          const float p1 = poly ? poly_exp2(x1) : fast_exp2(x1);
+          ps0 += p0;
+          ps1 += p1;
+          pk[i] = E::pack(p0, p1);
+        }
+        tc::tmem_st16u(lane_addr + (uint32_t)(c * 16), pk);
       }
-      l = l * alpha + psum;
-      // PV(j-1) must be done before O is rescaled (it writes O).
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(my_pv_done, (j - 1) & 1))) { failed = true; break; }
-      tc::fence_after_sync();
-      // P_j row r: 64 bf16 = 128 bytes, 128-byte swizzle (PV(j-1) has read P_{j-1})
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(my_p + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      // rescale O when a row's reference maximum moved (warp-uniform decision)
+      l = l * alpha + (ps0 + ps1);
+      // rescale O when a row's reference maximum moved (warp-uniform
+      // decision); P.V_tile(j-1) has completed (covered by s_full's commit),
+      // P.V_tile(j) waits for this warp's p_ready arrival
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {
@@ -467,12 +520,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tc::tmem_st32(lane_addr + kOCol + c * 32, o);
         }
       }
-      if (j > 0) tc::tmem_wait_st();
+      tc::tmem_wait_st();
       // V rows of keys past the context or of bad blocks become zero (once V_j
       // landed); tile 0 does it, before its p_ready, which the MMA warp awaits
       // before either tile's P.V(j).
       if (tile == 0 && (kb + kKeys > key_end || bad_mask)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (j / kStages) & 1))) { failed = true; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (uint32_t)((j / kStages) & 1)))) { failed = true; break; }
         uint8_t* v = stage_v(st);
         for (int i = r; i < kKeys * kChunks * 8; i += kRows) {
           const int c = i / (kKeys * 8), rem = i % (kKeys * 8);
@@ -481,15 +534,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             *reinterpret_cast<uint4*>(v + c * (kKeys * 128) + key * 128 + (rem % 8) * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();  // zeroed V rows -> visible to the tensor core
       }
-      fence_proxy_async_smem();  // P (and zeroed V rows) -> visible to the tensor core
       tc::fence_before_sync();
       mbar_arrive(&p_ready[tile]);
     }
     // ---- epilogue: O / l  ->  out (one partition) or fp32 partials
-    if (!failed && n_steps > 0 &&
-        !__all_sync(0xffffffffu, mbar_wait(my_pv_done, (n_steps - 1) & 1)))
-      failed = true;
+    if (!failed && n_steps > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done, 0))) failed = true;
     if (failed) {
       if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
     } else {
@@ -539,7 +590,105 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
 }
 
+// Longest-first order of the chunk kernel's work: the CTAs of a grid start in
+// index order, so listing the (sequence, tile pair, partition) items by
+// descending key steps makes the launch a longest-processing-time-first
+// schedule, and the last wave ends with short items. One CTA: a histogram of
+// the items' step counts (one bucket per thread), a descending scan, a
+// scatter. An item is listed exactly when the kernel would do work (or count
+// an error) for it; its step count is the kernel's n_steps.
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads)
+    chunk_plan_kernel(const int32_t* __restrict__ context_lens,
+                      const int32_t* __restrict__ q_start, int num_seqs, int num_q_tokens,
+                      int max_query_len, int max_context_len, int group, int part_blocks,
+                      int max_parts, uint2* __restrict__ items, int32_t* __restrict__ plan) {
+  __shared__ int hist[kPlanThreads];
+  __shared__ int cursor[kPlanThreads];
+  __shared__ int warp_sum[kPlanThreads / 32];
+  griddep_launch_dependents();  // the chunk kernel's CTAs may become resident now
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tok_per_tile = kRows / group;
+  // visit(s, f): f(local item index, steps) for every item of sequence s
+  auto visit = [&](int s, auto&& f) {
+    int L = context_lens[s];
+    L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
+    const int q0 = q_start[s];
+    int Tq = q_start[s + 1] - q0;
+    const bool bad_q = q0 < 0 || Tq < 0 || q0 + Tq > num_q_tokens;
+    if (!bad_q) Tq = min(Tq, min(L, max_query_len));
+    const int nblk = (L + 15) / 16;
+    const int n_parts = nblk > 0 ? (nblk + part_blocks - 1) / part_blocks : 1;
+    bool listed00 = false;
+    if (!bad_q) {
+      for (int t0 = 0, pair = 0; t0 < Tq; t0 += kTiles * tok_per_tile, ++pair) {
+        const int t_last = min(t0 + kTiles * tok_per_tile, Tq) - 1;
+        for (int p = 0; p < n_parts; ++p) {
+          const int kb = p * part_blocks * 16;
+          const int ke = min(min((p + 1) * part_blocks * 16, L), L - Tq + t_last + 1);
+          const int steps = ke > kb ? (ke - kb + kKeys - 1) / kKeys : 0;
+          f(pair * max_parts + p, steps);
+          listed00 |= pair == 0 && p == 0;
+        }
+      }
+    }
+    // The kernel counts a sequence's argument errors in its first item: keep
+    // that item even when it has no rows.
+    if (!listed00) f(0, 0);
+  };
+  hist[tid] = 0;
+  __syncthreads();
+  for (int s = tid; s < num_seqs; s += kPlanThreads)
+    visit(s, [&](int, int steps) { atomicAdd(&hist[min(steps, kPlanThreads - 1)], 1); });
+  __syncthreads();
+  // cursor[b] = items in buckets above b (more steps first)
+  const int b = kPlanThreads - 1 - tid;
+  const int v = hist[b];
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sum[lane] = w;
+  }
+  __syncthreads();
+  const int incl = x + (warp > 0 ? warp_sum[warp - 1] : 0);
+  cursor[b] = incl - v;
+  if (tid == kPlanThreads - 1) plan[0] = incl;
+  __syncthreads();
+  for (int s = tid; s < num_seqs; s += kPlanThreads)
+    visit(s, [&](int local, int steps) {
+      items[atomicAdd(&cursor[min(steps, kPlanThreads - 1)], 1)] =
+          make_uint2((unsigned)s, (unsigned)local);
+    });
+}
+
 }  // namespace
+
+bool prefill_tc_eligible(int32_t head_dim, int32_t group, int32_t max_query_len, int64_t parts,
+                         int32_t partition_tokens) {
+  const bool pow2 = group == 1 || group == 2 || group == 4 || group == 8 || group == 16;
+  return head_dim == kD && pow2 && (int64_t)max_query_len * group >= 64 &&
+         (parts <= 1 || partition_tokens % kKeys == 0);
+}
+
+int64_t prefill_tc_max_items(int32_t num_seqs, int32_t max_query_len, int32_t group,
+                             int64_t parts) {
+  const int64_t tiles = ((int64_t)max_query_len * group + kRows - 1) / kRows;
+  const int64_t pairs = (tiles + kTiles - 1) / kTiles;
+  return (int64_t)num_seqs * (pairs > 0 ? pairs : 1) * (parts > 0 ? parts : 1);
+}
 
 bool prefill_tc_supported(const DecodeLaunch& a) {
   const int g = a.group;
@@ -557,13 +706,42 @@ cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q,
     if (e != cudaSuccess) return e;
     const int qtiles = (a.max_query_len * a.group + kRows - 1) / kRows;
     const int pairs = (qtiles + kTiles - 1) / kTiles;
-    dim3 grid((unsigned)((int64_t)a.max_parts * pairs), a.num_kv_heads, a.num_seqs);
-    kern<<<grid, kThreadsTc, kSmemAlloc, stream>>>(
-        tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, a.q_start,
-        a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride, a.context_lens,
-        a.num_q_heads, a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
-        a.max_parts, a.dev_error);
-    return cudaGetLastError();
+    if (!a.chunk_plan) {
+      dim3 grid((unsigned)((int64_t)a.max_parts * pairs), a.num_kv_heads, a.num_seqs);
+      kern<<<grid, kThreadsTc, kSmemAlloc, stream>>>(
+          tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, a.q_start,
+          a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride, a.context_lens,
+          a.num_q_heads, a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
+          a.max_parts, a.dev_error, nullptr, nullptr, a.num_kv_heads);
+      return cudaGetLastError();
+    }
+    // Longest first: the plan kernel lists the items, the chunk kernel (a
+    // programmatic dependent: resident while the plan runs, reading nothing
+    // before griddepcontrol.wait) takes them in that order.
+    const int64_t n_max = prefill_tc_max_items(a.num_seqs, a.max_query_len, a.group,
+                                               a.max_parts) * a.num_kv_heads;
+    chunk_plan_kernel<<<1, kPlanThreads, 0, stream>>>(
+        a.context_lens, a.q_start, a.num_seqs, a.num_q_tokens, a.max_query_len,
+        a.max_context_len, a.group, a.part_blocks, a.max_parts, a.chunk_items, a.chunk_plan);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)n_max);
+    cfg.blockDim = dim3(kThreadsTc);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o,
+                              a.part_lse, a.q_start, a.num_q_tokens, a.max_query_len,
+                              a.block_tables, a.bt_stride, a.context_lens, a.num_q_heads,
+                              a.group, a.num_blocks, a.max_context_len, a.scale_log2,
+                              a.part_blocks, a.max_parts, a.dev_error,
+                              static_cast<const uint2*>(a.chunk_items),
+                              static_cast<const int32_t*>(a.chunk_plan), a.num_kv_heads);
   };
   return a.bf16 ? run((__nv_bfloat16*)nullptr) : run((__half*)nullptr);
 }

@@ -28,7 +28,8 @@ EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_bloc
            "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence",
            "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots", "pa_bm_append_slots",
            "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount", "pa_prefill_chunk",
-           "pa_decode_persistent_workspace_size", "pa_decode_persistent", "pa_read_probe")
+           "pa_decode_persistent_workspace_size", "pa_decode_persistent", "pa_read_probe",
+           "pa_prefill_chunk_workspace_size")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
                                            i32, i32, i64, i32, ctypes.c_float, i32, P, sz, P,
                                            ctypes.c_int, P]
             L.pa_prefill_chunk.restype = ctypes.c_int
+            L.pa_prefill_chunk_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32]
+            L.pa_prefill_chunk_workspace_size.restype = sz
             L.pa_decode_static.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                            i32, ctypes.c_float, i32, P, ctypes.c_int, P]
             L.pa_decode_static.restype = ctypes.c_int
@@ -176,6 +179,23 @@ def alloc_workspace(num_seqs, num_q_heads, head_dim, max_context_len, partition_
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
+def prefill_chunk_workspace_size(num_q_tokens: int, num_seqs: int, num_q_heads: int,
+                                 group_size: int, head_dim: int, max_query_len: int,
+                                 max_context_len: int, partition_tokens: int) -> int:
+    return int(lib().pa_prefill_chunk_workspace_size(num_q_tokens, num_seqs, num_q_heads,
+                                                     group_size, head_dim, max_query_len,
+                                                     max_context_len, partition_tokens))
+
+
+def alloc_chunk_workspace(num_q_tokens, num_seqs, num_q_heads, group_size, head_dim,
+                          max_query_len, max_context_len, partition_tokens,
+                          device) -> torch.Tensor | None:
+    """A workspace for pa_prefill_chunk with room for its longest-first plan."""
+    n = prefill_chunk_workspace_size(num_q_tokens, num_seqs, num_q_heads, group_size, head_dim,
+                                     max_query_len, max_context_len, partition_tokens)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
 def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
            block_tables: torch.Tensor, context_lens: torch.Tensor, *, scale: float,
            max_context_len: int, partition_tokens: int = 512,
@@ -224,7 +244,8 @@ def prefill_chunk(out: torch.Tensor, q: torch.Tensor, q_start: torch.Tensor, k_c
     if Hq % Hkv:
         raise ValueError("num_q_heads must be a multiple of num_kv_heads")
     if workspace is None:
-        workspace = alloc_workspace(T, Hq, D, max_context_len, partition_tokens, q.device)
+        workspace = alloc_chunk_workspace(T, S, Hq, Hq // Hkv, D, max_query_len, max_context_len,
+                                          partition_tokens, q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().pa_prefill_chunk(_ptr(out), _ptr(q), _ptr(q_start), T, int(max_query_len),
                                 _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),

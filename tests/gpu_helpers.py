@@ -63,15 +63,24 @@ class DeviceStep:
                   workspace=self.ws, dev_error=self.err)
         return out
 
-    def prefill(self, out=None):
-        """The chunk attention of a workload built by workloads.chunk_workload."""
+    def prefill(self, out=None, ordered=False):
+        """The chunk attention of a workload built by workloads.chunk_workload.
+        ordered=True gives pa_prefill_chunk the larger workspace of
+        pa_prefill_chunk_workspace_size, with which the tcgen05 path runs its
+        work longest first (a plan kernel); otherwise the partials' workspace
+        only (grid order)."""
         out = self.out if out is None else out
         w = self.w
         qs = torch.from_numpy(w.q_start).cuda()
+        mq = int(np.diff(w.q_start).max())
+        ws = self.ws
+        if ordered:
+            ws = pa.alloc_chunk_workspace(int(w.q.shape[0]), w.num_seqs, w.num_q_heads,
+                                          w.group_size, w.head_dim, mq, w.max_context_len,
+                                          self.P, "cuda")
         pa.prefill_chunk(out, self.q, qs, self.k_cache, self.v_cache, self.bt, self.cl,
-                         scale=w.scale, max_query_len=int(np.diff(w.q_start).max()),
-                         max_context_len=w.max_context_len, partition_tokens=self.P,
-                         workspace=self.ws, dev_error=self.err)
+                         scale=w.scale, max_query_len=mq, max_context_len=w.max_context_len,
+                         partition_tokens=self.P, workspace=ws, dev_error=self.err)
         return out
 
     def step(self):

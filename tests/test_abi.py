@@ -206,3 +206,23 @@ def test_read_probe_rejections(L):
     assert f(FAKE + 8, 1 << 20, 0, FAKE, None, None) == pa.PA_ERR_INVALID_ARG  # 16-byte base
     assert f(FAKE, (1 << 20) + 8, 1, FAKE, None, None) == pa.PA_ERR_INVALID_ARG  # 16-byte size
     assert f(FAKE, 0, 0, None, None, None) == pa.PA_OK                         # nothing to read
+
+
+def test_chunk_workspace_size(L):
+    """pa_prefill_chunk_workspace_size: the split partials of every query
+    row, plus -- on the tcgen05 path only -- 8 bytes per possible (sequence,
+    query-tile pair, partition) item and 256 bytes for the longest-first
+    plan."""
+    f, dws = L.pa_prefill_chunk_workspace_size, L.pa_decode_workspace_size
+    r256 = lambda x: -(-x // 256) * 256  # noqa: E731
+    # 16 sequences, 256-token chunks, group 4, D 128, no split: 1024 rows -> 8 tiles -> 4 pairs
+    assert f(4096, 16, 32, 4, 128, 256, 8192, 0) == 0 + r256(16 * 4 * 1 * 8) + 256
+    # split in 512-token partitions: 16 partitions of 8192 tokens
+    parts = 8192 // 512
+    assert f(4096, 16, 32, 4, 128, 256, 8192, 512) == \
+        dws(4096, 32, 128, 8192, 512) + r256(16 * 4 * parts * 8) + 256
+    # not the tcgen05 path: D 64, a partition size that is not a multiple of 128,
+    # too few rows -- the partials only
+    assert f(4096, 16, 32, 4, 64, 256, 8192, 512) == dws(4096, 32, 64, 8192, 512)
+    assert f(4096, 16, 32, 4, 128, 256, 8192, 64) == dws(4096, 32, 128, 8192, 64)
+    assert f(64, 16, 32, 4, 128, 4, 8192, 512) == dws(64, 32, 128, 8192, 512)

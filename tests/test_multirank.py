@@ -72,4 +72,4 @@ def test_single_rank_is_the_identity():
            "copy_ms": 0.125, "errors": 0}
     agg = bench.reduce_over_ranks(res, 1)
     assert agg == {"ms": 3.0, "e2e_ms": 0.0, "att_ms": 2.5, "write_ms": 0.25, "copy_ms": 0.125,
-                   "kv": float(w.kv_bytes()), "seqs": 5.0, "errors": 0}
+                   "sus_ms": 0.0, "kv": float(w.kv_bytes()), "seqs": 5.0, "errors": 0}
