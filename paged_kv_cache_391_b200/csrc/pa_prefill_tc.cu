@@ -89,32 +89,18 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA and integer pipes, for a share of the exponentials so that
-// the MUFU pipe (16 results per clock per SM, as few as the tensor core needs
-// at D = 128) is not the limit: x = n + f with n = round(x) (by adding
-// 1.5 * 2^23, which leaves n in the low mantissa bits) and f in [-0.5, 0.5];
-// 2^f by a cubic fitted here to minimise the relative error on that interval
-// (iteratively reweighted least squares over Chebyshev nodes: max relative
-// error 7.5e-5, below bf16's 2^-9 rounding of P); n is added to the exponent
-// field. Inputs below -126 give 0 (as ex2.approx.ftz does there).
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -127.f);
-  const float t = x + 12582912.f;          // 1.5 * 2^23: round x to an integer
-  const float f = x - (t - 12582912.f);    // in [-0.5, 0.5]
-  float p = fmaf(0.05517144f, f, 0.24261114f);
-  p = fmaf(p, f, 0.69326103f);
-  p = fmaf(p, f, 0.99992806f);
-  const int n = __float_as_int(t) - 0x4B400000;  // round(x), from the low mantissa bits
-  const float y = __int_as_float(__float_as_int(p) + (n << 23));
-  return x > -126.f ? y : 0.f;
+// Three-input max / min (one instruction on sm_100): the softmax is bound by
+// instruction issue, and its row-maximum reduction halves with them.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
-
-// Every kPolyEvery-th pair of exponentials of a row is taken by poly_exp2
-// (0: none).
-#ifndef PA_TC_POLY_EVERY
-#define PA_TC_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = PA_TC_POLY_EVERY;
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 // A row's running maximum is only moved (and O rescaled) when the new
 // maximum exceeds it by more than 2^8: until then P is taken against the
@@ -469,15 +455,33 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         cc = 1.f;
       } else {
-        float hi0 = s[0], lo0 = s[0], hi1 = s[1], lo1 = s[1];
+        // the largest logit is the largest raw score (the smallest, for a
+        // negative scale); four independent chains of three-input max
+        static_assert(kKeys % 8 == 4 || kKeys % 8 == 0, "reduction layout");
+        float e0 = s[0], e1 = s[1], e2 = s[2], e3 = s[3];
+        if (scale_log2 >= 0.f) {
 #pragma unroll
-        for (int i = 2; i < kKeys; i += 2) {
-          hi0 = fmaxf(hi0, s[i]);
-          lo0 = fminf(lo0, s[i]);
-          hi1 = fmaxf(hi1, s[i + 1]);
-          lo1 = fminf(lo1, s[i + 1]);
+          for (int i = 4; i + 8 <= kKeys; i += 8) {
+            e0 = max3(e0, s[i], s[i + 1]);
+            e1 = max3(e1, s[i + 2], s[i + 3]);
+            e2 = max3(e2, s[i + 4], s[i + 5]);
+            e3 = max3(e3, s[i + 6], s[i + 7]);
+          }
+          e0 = max3(e0, s[kKeys - 4], s[kKeys - 3]);
+          e1 = max3(e1, s[kKeys - 2], s[kKeys - 1]);
+          mx = max3(e0, e1, fmaxf(e2, e3)) * scale_log2;
+        } else {
+#pragma unroll
+          for (int i = 4; i + 8 <= kKeys; i += 8) {
+            e0 = min3(e0, s[i], s[i + 1]);
+            e1 = min3(e1, s[i + 2], s[i + 3]);
+            e2 = min3(e2, s[i + 4], s[i + 5]);
+            e3 = min3(e3, s[i + 6], s[i + 7]);
+          }
+          e0 = min3(e0, s[kKeys - 4], s[kKeys - 3]);
+          e1 = min3(e1, s[kKeys - 2], s[kKeys - 1]);
+          mx = min3(e0, e1, fminf(e2, e3)) * scale_log2;
         }
-        mx = (scale_log2 >= 0.f ? fmaxf(hi0, hi1) : fminf(lo0, lo1)) * scale_log2;
         cc = scale_log2;
       }
       float alpha = 1.f;
@@ -488,24 +492,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       const float m_use = m == -INFINITY ? 0.f : m;
       // P_j row r: 128 bf16 = 64 columns over the S columns already read
-      float ps0 = 0.f, ps1 = 0.f;
+      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;  // four chains of row-sum adds
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const bool poly = kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == 0;
-          const float x0 = fmaf(s[32 * c + 2 * i], cc, -m_use);
-          const float x1 = fmaf(s[32 * c + 2 * i + 1], cc, -m_use);
-          const float p0 = poly ? poly_exp2(x0) : fast_exp2(x0);
-          const float p1 = poly ? poly_exp2(x1) : fast_exp2(x1);
-          ps0 += p0;
-          ps1 += p1;
+          const float p0 = fast_exp2(fmaf(s[32 * c + 2 * i], cc, -m_use));
+          const float p1 = fast_exp2(fmaf(s[32 * c + 2 * i + 1], cc, -m_use));
+          if (i & 1) {
+            sa1 += p0;
+            sb1 += p1;
+          } else {
+            sa0 += p0;
+            sb0 += p1;
+          }
           pk[i] = E::pack(p0, p1);
         }
         tc::tmem_st16u(lane_addr + (uint32_t)(c * 16), pk);
       }
-      l = l * alpha + (ps0 + ps1);
+      l = l * alpha + ((sa0 + sa1) + (sb0 + sb1));
       // rescale O when a row's reference maximum moved (warp-uniform
       // decision); P.V_tile(j-1) has completed (covered by s_full's commit),
       // P.V_tile(j) waits for this warp's p_ready arrival
