@@ -73,3 +73,61 @@ def test_single_rank_is_the_identity():
     agg = bench.reduce_over_ranks(res, 1)
     assert agg == {"ms": 3.0, "e2e_ms": 0.0, "att_ms": 2.5, "write_ms": 0.25, "copy_ms": 0.125,
                    "sus_ms": 0.0, "kv": float(w.kv_bytes()), "seqs": 5.0, "errors": 0}
+
+
+def _shard_worker(rank, world, port, q):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bench
+    import oracle
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # each rank: its own shard of sequences, decoded with no exchange
+        w = bench.make_workload("gqa", 3, seed_offset=rank)
+        kc, vc = w.k_pool.copy(), w.v_pool.copy()
+        oracle.write_kv(w.new_k, w.new_v, kc, vc, w.slot_mapping)
+        out = oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, w.dtype)
+        got = [torch.zeros(out.size, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(got, torch.from_numpy(np.ascontiguousarray(out).reshape(-1)))
+        if rank == 0:
+            q.put([g.numpy() for g in got])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(240)
+def test_sequence_shards_need_no_exchange():
+    """The data-parallel split: each rank decodes its own sequences; the
+    whole job's output is the concatenation of the ranks' outputs, each equal
+    to a single process decoding that shard, and the shards differ."""
+    import numpy as np
+
+    import bench
+    import oracle
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.SimpleQueue()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    gathered = q.get()          # before joining: the result does not fit in the pipe's buffer
+    for p in procs:
+        p.join(200)
+        assert p.exitcode == 0
+    for r in range(world):
+        w = bench.make_workload("gqa", 3, seed_offset=r)
+        kc, vc = w.k_pool.copy(), w.v_pool.copy()
+        oracle.write_kv(w.new_k, w.new_v, kc, vc, w.slot_mapping)
+        want = oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, w.dtype)
+        assert np.array_equal(gathered[r], want.reshape(-1))
+    assert not np.array_equal(gathered[0], gathered[1])
