@@ -602,7 +602,7 @@ def run_gpu(args, name, rank, world, device, probe_buf=None, e2e_on=True):
             "write_ms": write_ms, "copy_ms": copy_ms, "copy_pairs": int(len(copy_pairs_t)),
             "copy_what": copy_what, "short_reps": short_reps, "rounds": rounds,
             "errors": errors, "e2e": e2e, "launches": launches_per_step,
-            "persistent": persistent}
+            "persistent": persistent, "tc_path": tc_path}
 
 
 def l2_note(w) -> str:
@@ -837,6 +837,8 @@ def workload_record(name, res, agg, args, world, ceiling) -> dict:
                      else "write_kv + attention") + " (partitions + LSE reduce when split)",
             "scheduler": ("persistent: plan kernel + work-queue grid of SMs x resident CTAs"
                           if res["persistent"] else
+                          "longest first: plan kernel + one CTA per (query-tile pair, partition, "
+                          "KV head, sequence) in descending key count" if res.get("tc_path") else
                           "grid: one CTA per (partition, KV head, sequence)"),
             "accumulate": "fp32",
             "l2": l2_note(w),
