@@ -392,7 +392,12 @@ int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
  *             every resident thread sweeping the buffer;
  *   method 1: bulk asynchronous copies (cp.async.bulk, 16 KiB, no multicast)
  *             into a shared-memory ring per CTA -- the engine the decode
- *             kernels read their tiles with.
+ *             kernels read their tiles with;
+ *   method 2: the paged decode's access pattern without its arithmetic: the
+ *             buffer as 4 KiB tiles (one KV head of one cache block at
+ *             D = 128), each read once in a scattered order by two 2 KiB TMA
+ *             tensor boxes, in the decode kernel's CTA shape (reads
+ *             floor(bytes / 8 KiB) * 8 KiB bytes) -- the paged-read ceiling.
  * Each CTA XORs a fold of what it read into *sink (device uint64, 8-byte
  * aligned; its value means nothing, it only keeps the loads alive). A bulk
  * wait that gives up adds PA_DEV_ERR_TIMEOUT to *dev_error (nullable). Time

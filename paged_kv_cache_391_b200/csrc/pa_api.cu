@@ -450,11 +450,28 @@ pa_status pa_swap_blocks(void* const* src_k, void* const* src_v, void* const* ds
 
 pa_status pa_read_probe(const void* buf, size_t bytes, int32_t method, uint64_t* sink,
                         int32_t* dev_error, void* stream) {
-  if (method != 0 && method != 1) return PA_ERR_INVALID_ARG;
+  if (method < 0 || method > 2) return PA_ERR_INVALID_ARG;
   if (bytes == 0) return PA_OK;
   if (!buf || !sink || !aligned(buf, 16) || bytes % 16 || !aligned(sink, 8) ||
       (dev_error && !aligned(dev_error, 4)))
     return PA_ERR_INVALID_ARG;
+  if (method == 2) {
+    // whole 4 KiB tiles, an even number of them (two per stage)
+    const int64_t n_tiles = (int64_t)(bytes / 4096) & ~(int64_t)1;
+    if (n_tiles < 2 || n_tiles > (int64_t(1) << 31)) return PA_ERR_INVALID_ARG;
+    CUtensorMap tm;
+    pa_status st = encode_pool_map(&tm, buf, n_tiles, 1, 128, PA_DTYPE_BF16);
+    if (st != PA_OK) return st;
+    // a stride near n / golden ratio, coprime with n: consecutive reads land
+    // far apart, and every tile is read once
+    int64_t stride = (int64_t)((double)n_tiles * 0.6180339887) | 1;
+    auto gcd = [](int64_t a, int64_t b) { while (b) { const int64_t t = a % b; a = b; b = t; } return a; };
+    while (gcd(stride, n_tiles) != 1) stride += 2;
+    cudaError_t e = pa::launch_read_probe_scattered(
+        tm, n_tiles, stride % n_tiles, n_tiles / 3, reinterpret_cast<unsigned long long*>(sink),
+        dev_error, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : cuda_fail(e);
+  }
   cudaError_t e = pa::launch_read_probe(buf, bytes, method,
                                         reinterpret_cast<unsigned long long*>(sink), dev_error,
                                         static_cast<cudaStream_t>(stream));

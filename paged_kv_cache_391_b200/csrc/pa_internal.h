@@ -90,5 +90,10 @@ cudaError_t launch_block_copy(void* const* src_k, void* const* src_v, void* cons
 // Streaming-read probe (pa_read_probe): method 0 = vector loads, 1 = bulk copies.
 cudaError_t launch_read_probe(const void* buf, size_t bytes, int method,
                               unsigned long long* sink, int32_t* dev_error, cudaStream_t stream);
+// Method 2: n_tiles 4 KiB tiles of `tm` (a [n][1][16][128] 16-bit pool map)
+// read in the order (i * stride + offset) mod n_tiles.
+cudaError_t launch_read_probe_scattered(const CUtensorMap& tm, int64_t n_tiles, int64_t stride,
+                                        int64_t offset, unsigned long long* sink,
+                                        int32_t* dev_error, cudaStream_t stream);
 
 }  // namespace pa

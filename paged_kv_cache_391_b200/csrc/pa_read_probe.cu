@@ -10,6 +10,8 @@
 //   method 1: bulk asynchronous copies (cp.async.bulk, no multicast) of 16 KiB
 //             chunks into a 6-stage shared-memory ring per CTA, mbarrier
 //             tracked -- the same engine the decode kernels read tiles with.
+//   method 2: scattered 4 KiB tiles by 2 KiB TMA tensor boxes, in the decode
+//             kernel's CTA shape (the paged-read ceiling; below).
 // One atomic XOR per CTA into *sink. All waits are bounded.
 #include "pa.h"
 #include "pa_device.cuh"
@@ -139,7 +141,98 @@ __global__ void __launch_bounds__(32)
   atomicXor(sink, (unsigned long long)acc);
 }
 
+// Method 2: the paged decode's access pattern without its arithmetic. The
+// buffer is n 4 KiB tiles (16 rows of 256 bytes, like one KV head of one cache
+// block at D = 128); global tile i is read at tile (i * stride + offset) mod n
+// (stride coprime with n: every tile once, scattered), as two 2 KiB TMA boxes
+// with the 128-byte swizzle, two tiles per stage, in the decode CTA's shape:
+// 4 warps, each with a 2-stage ring, 3 CTAs per SM. Every wait is bounded.
+constexpr int kScatWarps = 4;
+constexpr int kScatStages = 2;
+constexpr int kScatStageBytes = 8192;  // two tiles
+constexpr int kScatSmem = kScatWarps * kScatStages * kScatStageBytes + 1024;
+
+__global__ void __launch_bounds__(kScatWarps * 32)
+    read_scattered_kernel(const __grid_constant__ CUtensorMap tm, int64_t n_tiles,
+                          int64_t stride, int64_t offset, unsigned long long* sink,
+                          int32_t* dev_error) {
+  extern __shared__ uint8_t raw[];
+  __shared__ uint64_t bars[kScatWarps * kScatStages];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t* ring = base + warp * kScatStages * kScatStageBytes;
+  uint64_t* wb = bars + warp * kScatStages;
+  // this warp's pairs of tiles: p = gw, gw + nw, ... (pair p = tiles 2p, 2p+1)
+  const int64_t gw = (int64_t)blockIdx.x * kScatWarps + warp;
+  const int64_t nw = (int64_t)gridDim.x * kScatWarps;
+  const int64_t n_pairs = n_tiles / 2;
+  const int64_t mine = gw < n_pairs ? (n_pairs - 1 - gw) / nw + 1 : 0;
+  if (lane == 0) {
+    for (int st = 0; st < kScatStages; ++st) mbar_init(&wb[st], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  auto tile_of = [&](int64_t i) { return (int)((i * stride + offset) % n_tiles); };
+  auto issue = [&](int64_t k) {  // lane 0
+    const int st = (int)(k % kScatStages);
+    uint8_t* dst = ring + st * kScatStageBytes;
+    const int64_t p = gw + k * nw;
+    mbar_arrive_expect_tx(&wb[st], kScatStageBytes);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int tile = tile_of(2 * p + t);
+      tma_load_4d(dst + t * 4096, &tm, &wb[st], 0, 0, 0, tile);
+      tma_load_4d(dst + t * 4096 + 2048, &tm, &wb[st], 64, 0, 0, tile);
+    }
+  };
+  if (lane == 0)
+    for (int64_t k = 0; k < mine && k < kScatStages; ++k) issue(k);
+  uint32_t acc = 0;
+  int64_t k = 0;
+  bool failed = false;
+  for (; k < mine; ++k) {
+    const int st = (int)(k % kScatStages);
+    if (!__all_sync(0xffffffffu, mbar_wait(&wb[st], (uint32_t)((k / kScatStages) & 1)))) {
+      failed = true;
+      break;
+    }
+    acc ^= *reinterpret_cast<const uint32_t*>(ring + st * kScatStageBytes + lane * 256);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && k + kScatStages < mine) issue(k + kScatStages);
+  }
+  if (failed) {
+    // Let the copies in flight land (each wait bounded) before the CTA exits.
+    const int64_t last = k + kScatStages < mine ? k + kScatStages : mine;
+    for (int64_t j = k; j < last; ++j)
+      (void)mbar_wait(&wb[j % kScatStages], (uint32_t)((j / kScatStages) & 1));
+    if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
+  }
+  fold_into_sink(acc, sink);
+}
+
 }  // namespace
+
+cudaError_t launch_read_probe_scattered(const CUtensorMap& tm, int64_t n_tiles, int64_t stride,
+                                        int64_t offset, unsigned long long* sink,
+                                        int32_t* dev_error, cudaStream_t stream) {
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  e = cudaFuncSetAttribute(read_scattered_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kScatSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, read_scattered_kernel,
+                                                    kScatWarps * 32, kScatSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = sms * (per_sm > 0 ? per_sm : 1);
+  read_scattered_kernel<<<grid, kScatWarps * 32, kScatSmem, stream>>>(tm, n_tiles, stride, offset,
+                                                                      sink, dev_error);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_read_probe(const void* buf, size_t bytes, int method,
                               unsigned long long* sink, int32_t* dev_error,

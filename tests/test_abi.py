@@ -200,7 +200,8 @@ def test_read_probe_rejections(L):
     """pa_read_probe refuses bad methods, pointers, alignment and sizes on
     the host, before any launch."""
     f = L.pa_read_probe
-    assert f(FAKE, 1 << 20, 2, FAKE, None, None) == pa.PA_ERR_INVALID_ARG      # method
+    assert f(FAKE, 1 << 20, 3, FAKE, None, None) == pa.PA_ERR_INVALID_ARG      # method
+    assert f(FAKE, 4096, 2, FAKE, None, None) == pa.PA_ERR_INVALID_ARG         # < two tiles
     assert f(None, 1 << 20, 0, FAKE, None, None) == pa.PA_ERR_INVALID_ARG      # buffer
     assert f(FAKE, 1 << 20, 0, None, None, None) == pa.PA_ERR_INVALID_ARG      # sink
     assert f(FAKE + 8, 1 << 20, 0, FAKE, None, None) == pa.PA_ERR_INVALID_ARG  # 16-byte base
