@@ -110,3 +110,31 @@ def test_tensor_core_tile_pairs(P):
     w = W.chunk_workload("pairs", [300, 1000, 2500], [96, 160, 288], num_q_heads=8,
                          num_kv_heads=2, head_dim=128, dtype="bf16", seed=50 + P)
     _check(w, P)
+
+
+@pytest.mark.parametrize("name", ["chunked_prefill", "spec_verify"])
+def test_full_size_sampled(name):
+    """The two query-chunk workloads at full size, in the launch configuration
+    the benchmark times (the chunk workspace, so the tcgen05 path runs its
+    longest-first plan): pools bit-exact after the step's writes; outputs on
+    sampled rows plus every head of the first and last query token of the
+    shortest and the longest sequence."""
+    w = W.CONFIGS[name]()
+    d = DeviceStep(w)
+    d.cache_ops()
+    d.prefill(ordered=True)
+    torch.cuda.synchronize()
+    kc, vc = oracle_caches_after_step(w)
+    assert np.array_equal(host16(d.k_cache), kc) and np.array_equal(host16(d.v_cache), vc)
+    T, Hq = int(w.q.shape[0]), w.num_q_heads
+    rng = np.random.default_rng(31)
+    rows = set(rng.choice(T * Hq, size=48, replace=False).tolist())
+    for s in (int(np.argmin(w.context_lens)), int(np.argmax(w.context_lens))):
+        for tok in (int(w.q_start[s]), int(w.q_start[s + 1]) - 1):
+            rows.update(range(tok * Hq, (tok + 1) * Hq))
+    rows = np.array(sorted(rows), np.int64)
+    ref = oracle.prefill_chunk(w.q, w.q_start, kc, vc, w.block_tables, w.context_lens, w.scale,
+                               w.dtype, rows=rows)
+    gpu = to_f64(d.out).reshape(T * Hq, -1)[rows]
+    assert_decode_close(gpu, ref, name)
+    assert int(d.err.item()) == 0
