@@ -191,14 +191,15 @@ __device__ __forceinline__ bool attend_item(const ItemArgs<T>& A, uint8_t* smem,
   }
 
   // Physical block ids, 32 iterations per register window; ids outside the
-  // pool are counted once (by the KV-head-0 CTA) and skipped.
+  // pool are skipped and counted once (by the KV-head-0 CTA of the first
+  // query tile: every query tile's CTA reads the partition's whole table).
   const int32_t* bt_mine = block_tables + (size_t)seq * bt_stride + blk_begin + warp;
   auto load_pid = [&](int it) -> int {
     int p = -1;
     if (it < n_mine) {
       p = __ldg(bt_mine + kWarps * it);
       if (p < 0 || p >= num_blocks) {
-        if (kvh == 0 && dev_error) atomicAdd(dev_error, 1);
+        if (kvh == 0 && qtile == 0 && dev_error) atomicAdd(dev_error, 1);
         p = -1;
       }
     }

@@ -234,12 +234,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // its "empty" barrier; the loads run up to kStages steps ahead.
     const int lb_first = key_begin / 16;
     const int nblk_keys = (key_end - key_begin + 15) / 16;
+    // A table entry outside the pool is skipped (not loaded; the softmax
+    // masks its keys) and counted once: by the KV-head-0 CTA of the last
+    // pair of query tiles, whose causal horizon covers the whole partition.
+    const bool count_bad =
+        dev_error && kvh == 0 && t0 + kTiles * tok_per_tile >= Tq;
     auto load_window = [&](int w) {
       const int i = 32 * w + lane;
       int p = -1;
       if (i < nblk_keys) {
         p = __ldg(bt_row + lb_first + i);
-        if (p < 0 || p >= num_blocks) p = -1;
+        if (p < 0 || p >= num_blocks) {
+          if (count_bad) atomicAdd(dev_error, 1);
+          p = -1;
+        }
       }
       return p;
     };

@@ -218,6 +218,12 @@ def test_decode_bad_table_entry_is_counted_and_skipped():
     kc, vc = oracle_caches_after_step(w)
     ref = oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, w.dtype)
     assert_decode_close(out[1], ref[1])
+    # skipping a full block is attention over the other tokens, and attention
+    # does not depend on the order of its keys: the oracle over the table with
+    # that entry deleted and the context 16 tokens shorter
+    bt0 = np.delete(w.block_tables[0], 1)[None, :]
+    ref0 = oracle.decode(w.q[:1], kc, vc, bt0, np.array([24], np.int32), w.scale, w.dtype)
+    assert_decode_close(out[:1], ref0, "skipped block")
 
 
 def test_context_longer_than_max_is_clamped_and_counted():

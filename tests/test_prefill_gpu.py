@@ -138,3 +138,38 @@ def test_full_size_sampled(name):
     gpu = to_f64(d.out).reshape(T * Hq, -1)[rows]
     assert_decode_close(gpu, ref, name)
     assert int(d.err.item()) == 0
+
+
+@pytest.mark.parametrize("D,dtype,P", [(128, "bf16", 0), (128, "bf16", 512), (64, "f16", 512)])
+def test_bad_table_entry_in_a_chunk_is_skipped_and_counted_once(D, dtype, P):
+    """A table entry outside the pool, before the chunk: the block is skipped
+    (the tcgen05 path at D 128, the mma.sync path at D 64) and counted once
+    however many query tiles read it; the result is the oracle's over the
+    table with that entry deleted and the context 16 tokens shorter (the
+    order of keys does not matter to attention)."""
+    w = W.chunk_workload("badchunk", [900, 1200], [200, 96], num_q_heads=8, num_kv_heads=2,
+                         head_dim=D, dtype=dtype, seed=61 + D + P)
+    d = DeviceStep(w, P)
+    d.cache_ops()
+    bt = d.bt.clone()
+    bt[0, 10] = w.num_blocks + 7          # tokens 160..175 of sequence 0, before its chunk
+    qs = torch.from_numpy(w.q_start).cuda()
+    for ordered in (False, True):
+        d.err.zero_()
+        out = torch.full_like(d.out, float("nan"))
+        mq = int(np.diff(w.q_start).max())
+        ws = (pa.alloc_chunk_workspace(int(w.q.shape[0]), w.num_seqs, w.num_q_heads,
+                                       w.group_size, D, mq, w.max_context_len, P, "cuda")
+              if ordered else d.ws)
+        pa.prefill_chunk(out, d.q, qs, d.k_cache, d.v_cache, bt, d.cl, scale=w.scale,
+                         max_query_len=mq, max_context_len=w.max_context_len,
+                         partition_tokens=P, workspace=ws, dev_error=d.err)
+        torch.cuda.synchronize()
+        assert int(d.err.item()) == 1
+        kc, vc = oracle_caches_after_step(w)
+        bt_ref = w.block_tables.copy()
+        bt_ref[0, 10:-1] = w.block_tables[0, 11:]
+        lens = w.context_lens.copy()
+        lens[0] -= 16
+        ref = oracle.prefill_chunk(w.q, w.q_start, kc, vc, bt_ref, lens, w.scale, w.dtype)
+        assert_decode_close(to_f64(out), ref, f"skipped block, ordered={ordered}")
