@@ -58,9 +58,10 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
 
 
 # Test-only builds of the same sources with extra defines. "waittest": every
-# K/V tile wait of the decode kernels probes once (PA_TEST_TILE_WAIT_ONCE), so
-# tests can make a bounded wait run out without withholding any copy.
-VARIANTS = {"waittest": ["-DPA_TEST_TILE_WAIT_ONCE"]}
+# K/V tile wait of the decode kernels reports at once that it ran out of time
+# (PA_TEST_TILE_WAIT_EXPIRED), so tests take the timeout path without
+# withholding any copy.
+VARIANTS = {"waittest": ["-DPA_TEST_TILE_WAIT_EXPIRED"]}
 
 
 def variant_path(name: str) -> str:

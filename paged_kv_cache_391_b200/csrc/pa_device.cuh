@@ -76,27 +76,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// One non-blocking probe of the phase with the given parity.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // The wait of the decode kernels on a K/V tile. A build for testing the
-// timeout path defines PA_TEST_TILE_WAIT_ONCE: a tile wait then probes once
-// and gives up unless its copy has landed (the drain that follows still
-// waits up to kWaitLimitNs for every copy in flight). Product builds wait up
-// to kWaitLimitNs.
+// timeout path defines PA_TEST_TILE_WAIT_EXPIRED: every tile wait then reports
+// that it ran out of time at once, before looking at the barrier, as a real
+// wait does after kWaitLimitNs; the drain that follows still waits up to
+// kWaitLimitNs for every copy in flight. Product builds wait up to
+// kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait_tile(uint64_t* bar, uint32_t parity) {
-#ifdef PA_TEST_TILE_WAIT_ONCE
-  return mbar_test_wait(bar, parity);
+#ifdef PA_TEST_TILE_WAIT_EXPIRED
+  (void)bar;
+  (void)parity;
+  return false;
 #else
   return mbar_wait(bar, parity);
 #endif
