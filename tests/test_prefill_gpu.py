@@ -173,3 +173,15 @@ def test_bad_table_entry_in_a_chunk_is_skipped_and_counted_once(D, dtype, P):
         lens[0] -= 16
         ref = oracle.prefill_chunk(w.q, w.q_start, kc, vc, bt_ref, lens, w.scale, w.dtype)
         assert_decode_close(to_f64(out), ref, f"skipped block, ordered={ordered}")
+
+
+@pytest.mark.parametrize("Hq,Hkv,dtype", [(8, 4, "bf16"), (8, 4, "f16"), (8, 2, "f16"),
+                                          (16, 1, "f16"), (4, 4, "f16")])
+@pytest.mark.parametrize("P", [0, 256])
+def test_tensor_core_groups_and_fp16(Hq, Hkv, dtype, P):
+    """The tcgen05 path (D 128, a power-of-two group, enough rows) with fp16
+    operands as well as bf16, and at group 2: ragged chunks over several
+    partitions, in grid and longest-first order (both checked by _check)."""
+    w = W.chunk_workload("tcg", [700, 1500, 260], [120, 64, 260], num_q_heads=Hq,
+                         num_kv_heads=Hkv, head_dim=128, dtype=dtype, seed=Hq * 3 + Hkv + P)
+    _check(w, P)
