@@ -207,9 +207,12 @@ pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
  *                   with >= pa_prefill_chunk_workspace_size(...) bytes
  *                   (256-byte aligned), a plan kernel first lists the work
  *                   items by descending key count in the space after the
- *                   partials and the chunk kernel takes them in that order
- *                   (longest first; fewer idle SMs in the last wave); with
- *                   less it runs in grid order. Same result either way.
+ *                   partials, with a work counter, and the chunk kernel runs
+ *                   one CTA per SM, each taking the next item of that list
+ *                   whenever it is ready for one (longest first; no per-item
+ *                   launch and set-up cost, fewer idle SMs at the end); with
+ *                   less it runs one CTA per item in grid order. Same result
+ *                   either way, bit for bit.
  *   other arguments as for pa_decode. A sequence whose query range falls
  *   outside [0, num_q_tokens) is skipped, one whose Tq exceeds max_query_len
  *   or its context length is clamped; both are counted in dev_error. With a
@@ -219,7 +222,8 @@ pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
 /* Workspace bytes for pa_prefill_chunk's longest-first order: the split
  * partials (pa_decode_workspace_size of num_q_tokens rows) plus, when the call
  * takes the tcgen05 path, 8 bytes per possible (sequence, query-tile pair,
- * partition) item and 256 bytes. 0 if no workspace is needed. */
+ * partition) item and 256 bytes (item count and work counter). 0 if no
+ * workspace is needed. */
 size_t pa_prefill_chunk_workspace_size(int32_t num_q_tokens, int32_t num_seqs,
                                        int32_t num_q_heads, int32_t group_size, int32_t head_dim,
                                        int32_t max_query_len, int32_t max_context_len,

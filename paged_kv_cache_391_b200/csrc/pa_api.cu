@@ -309,7 +309,7 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
                                          partition_tokens);
     if (plan && workspace && aligned(workspace, 256) && workspace_bytes >= need + plan &&
         pa::prefill_tc_max_items(num_seqs, max_query_len, group_size, parts) * num_kv_heads <=
-            0x7fffffff) {
+            0x7fffffff - 65536) {  // the work counter passes the item count by one per CTA
       char* tail = static_cast<char*>(workspace) + need;
       const int64_t items = pa::prefill_tc_max_items(num_seqs, max_query_len, group_size, parts);
       a.chunk_items = reinterpret_cast<uint2*>(tail);

@@ -8,14 +8,17 @@
 // With many query rows per KV head this is a dense contraction, so it runs on
 // tcgen05 instead of the 16-row mma.sync tiles of the decode kernel.
 //
-// One CTA per (pair of 128-row query tiles, partition, KV head, sequence);
-// tile rows are (query token, head) pairs of the KV head's query group. Both
-// tiles share every K/V tile the CTA loads. 320 threads, one CTA per SM:
+// A work item is a (pair of 128-row query tiles, partition, KV head,
+// sequence); tile rows are (query token, head) pairs of the KV head's query
+// group. Both tiles share every K/V tile loaded for the item. Without a plan
+// one CTA runs one item (grid order); with the plan (longest first) one CTA
+// per SM runs items from a work counter until the list is exhausted, keeping
+// its TMEM, barriers and rings across items. 320 threads, one CTA per SM:
 //  * warps 0-3 and 4-7: softmax of tile 0 and tile 1. Thread r of a
 //    warpgroup owns row r of its tile: TMEM lane r of its S, P and O.
-//  * warp 8: TMA loads (Q once; per step K and V of 8 cache blocks = 128
-//    keys, each in its own 2-stage ring, sixteen lanes issuing a ring's
-//    sixteen boxes).
+//  * warp 8: TMA loads (per step K and V of 8 cache blocks = 128 keys, each in
+//    its own 2-stage ring, sixteen lanes issuing a ring's sixteen boxes; an
+//    item's Q after its first K and V) and, with the plan, the next item.
 //  * warp 9, one lane: every MMA:
 //      S_i(j)  = Q_i K_j^T      (M=128, N=128 keys, K=D; Q, K K-major in smem)
 //      O_i    += P_i(j) V_j     (M=128, N=D, K=128 keys; P in TMEM, V MN-major
@@ -73,9 +76,11 @@ constexpr int kKOff = kTiles * kQBytes;            // K stages
 constexpr int kVOff = kKOff + kStages * kKBytes;   // V stages
 constexpr int kBarOff = kVOff + kStages * kVBytes;
 // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2],
-// s_full[2 tiles], p_ready[2 tiles], o_done, mma_drain; then the TMEM address
-constexpr int kNumBars = 1 + 4 * kStages + 2 * kTiles + 2;
-constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+// s_full[2 tiles], p_ready[2 tiles], o_done, mma_drain, q_empty,
+// item_full[2], item_empty[2]; then the two item slots and the TMEM address
+constexpr int kNumBars = 1 + 4 * kStages + 2 * kTiles + 2 + 1 + 4;
+constexpr int kItemSlotOff = kBarOff + kNumBars * 8;
+constexpr int kTmemSlotOff = kItemSlotOff + 8;
 constexpr int kSmemBytes = kTmemSlotOff + 16;
 // The dynamic shared memory is declared 1024-byte aligned and the kernel
 // checks it (no slack is reserved).
@@ -108,6 +113,75 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
 // representable in bf16), and O / l is unchanged by the choice of reference.
 constexpr float kRescaleLog2 = 8.f;
 
+// One unit of the chunk kernel's work: a pair of query tiles of one
+// sequence's chunk, one partition of its keys, one KV head; and what every
+// role derives from it (uniform over the CTA).
+struct ChunkItem {
+  int seq, kvh, part, qtile;  // qtile: the pair's first tile
+  int L, q0, Tq, t0, n_parts, key_begin, key_end, n_steps;
+  bool skip;                  // no rows or no keys of this item exist
+  int err_count;              // argument errors this item counts (its first item only)
+};
+
+__device__ __forceinline__ ChunkItem chunk_item(int seq, int kvh, int part, int qtile,
+                                                const int32_t* __restrict__ q_start,
+                                                int num_q_tokens, int max_query_len,
+                                                const int32_t* __restrict__ context_lens,
+                                                int group, int max_context_len, int part_blocks) {
+  ChunkItem it;
+  it.seq = seq;
+  it.kvh = kvh;
+  it.part = part;
+  it.qtile = qtile;
+  it.err_count = 0;
+  it.skip = false;
+  const bool counts = part == 0 && kvh == 0 && qtile == 0;
+  int L = context_lens[seq];
+  if (L < 0 || L > max_context_len) {
+    it.err_count += counts;
+    L = L < 0 ? 0 : max_context_len;
+  }
+  it.L = L;
+  it.q0 = q_start[seq];
+  int Tq = q_start[seq + 1] - it.q0;
+  it.n_steps = 0;
+  it.t0 = 0;
+  it.n_parts = 1;
+  it.key_begin = it.key_end = 0;
+  if (it.q0 < 0 || Tq < 0 || it.q0 + Tq > num_q_tokens) {
+    it.err_count += counts;
+    it.Tq = 0;
+    it.skip = true;
+    return it;
+  }
+  if (Tq > min(L, max_query_len)) {
+    it.err_count += counts;
+    Tq = min(L, max_query_len);
+  }
+  it.Tq = Tq;
+  const int tok_per_tile = kRows / group;
+  it.t0 = qtile * tok_per_tile;
+  const int nblk_seq = (L + 15) / 16;
+  it.n_parts = nblk_seq > 0 ? (nblk_seq + part_blocks - 1) / part_blocks : 1;
+  if (it.t0 >= Tq || part >= it.n_parts) {
+    it.skip = true;
+    return it;
+  }
+  it.key_begin = part * part_blocks * 16;
+  const int t_last = min(it.t0 + kTiles * tok_per_tile, Tq) - 1;  // the pair's last query token
+  // keys the pair can see in this partition: up to the last row's causal limit
+  it.key_end = min(min((part + 1) * part_blocks * 16, L), L - Tq + t_last + 1);
+  it.n_steps = it.key_end > it.key_begin ? (it.key_end - it.key_begin + kKeys - 1) / kKeys : 0;
+  return it;
+}
+
+// Grid mode runs the one item its block index names. Plan mode is persistent:
+// one CTA per SM, each taking items of the plan's list (longest first) from a
+// work counter until the list is exhausted. The TMA warp takes the next item
+// once it has issued every load of the current one and posts it in a
+// two-slot ring (item_full / item_empty) for the MMA and softmax warps; so the
+// next item's Q and first K / V loads overlap the current item's end, and the
+// TMEM allocation, the barriers and their phases carry over between items.
 template <typename T>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -119,7 +193,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                       const int32_t* __restrict__ context_lens, int num_q_heads, int group,
                       int64_t num_blocks, int max_context_len, float scale_log2,
                       int part_blocks, int max_parts, int32_t* __restrict__ dev_error,
-                      const uint2* __restrict__ items, const int32_t* __restrict__ plan,
+                      const uint2* __restrict__ items, int32_t* __restrict__ plan,
                       int num_kv_heads) {
   using E = Elem<T>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -132,65 +206,48 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint64_t* v_empty = v_full + kStages;             // [stage]
   uint64_t* s_full = v_empty + kStages;             // [tile]
   uint64_t* p_ready = s_full + kTiles;              // [tile]
-  uint64_t* o_done = p_ready + kTiles;
+  uint64_t* o_done = p_ready + kTiles;              // an item's O final
   uint64_t* mma_drain = o_done + 1;                 // failure path only
+  uint64_t* q_empty = mma_drain + 1;                // an item's last S MMAs done: Q reusable
+  uint64_t* item_full = q_empty + 1;                // [2] plan mode: an item posted
+  uint64_t* item_empty = item_full + 2;             // [2] plan mode: an item read by all roles
+  int32_t* item_slot = reinterpret_cast<int32_t*>(smem + kItemSlotOff);  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlotOff);
 
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (smem_addr(smem) & 1023) {  // the 128-byte swizzle needs 1024-byte aligned tiles
-    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && dev_error)
+    if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && dev_error)
       atomicAdd(dev_error, 1);
     return;
   }
-  // The CTA's work: (pair of query tiles, partition, KV head, sequence) from
-  // the grid, or -- longest first -- from the plan (a 1-D grid; item w / H_kv
-  // of the plan's list, KV head w % H_kv).
-  int kvh, seq, part, qtile;
-  if (plan) {
-    griddep_wait();  // the plan kernel's list is complete and visible
-    const int64_t w = blockIdx.x;
-    if (w >= (int64_t)plan[0] * num_kv_heads) return;
-    const uint2 it = items[w / num_kv_heads];
-    kvh = (int)(w % num_kv_heads);
-    seq = (int)it.x;
-    part = (int)(it.y % (unsigned)max_parts);
-    qtile = (int)(it.y / (unsigned)max_parts) * kTiles;
+  // The item with index w into the plan's list x KV heads, or (kGridItem) the
+  // one the block index names. Recomputed where needed rather than kept.
+  constexpr int kGridItem = -2;
+  auto item_of = [&](int w) {
+    int seq, kvh, part, qtile;
+    if (w == kGridItem) {
+      seq = blockIdx.z;
+      kvh = blockIdx.y;
+      part = (int)(blockIdx.x % (unsigned)max_parts);
+      qtile = (int)(blockIdx.x / (unsigned)max_parts) * kTiles;
+    } else {
+      const uint2 pi = items[w / num_kv_heads];
+      seq = (int)pi.x;
+      kvh = w % num_kv_heads;
+      part = (int)(pi.y % (unsigned)max_parts);
+      qtile = (int)(pi.y / (unsigned)max_parts) * kTiles;
+    }
+    return chunk_item(seq, kvh, part, qtile, q_start, num_q_tokens, max_query_len,
+                      context_lens, group, max_context_len, part_blocks);
+  };
+  const bool persistent = plan != nullptr;
+  if (persistent) {
+    griddep_wait();  // the plan kernel's list and zeroed counter are complete and visible
   } else {
-    kvh = blockIdx.y;
-    seq = blockIdx.z;
-    part = (int)(blockIdx.x % (unsigned)max_parts);
-    qtile = (int)(blockIdx.x / (unsigned)max_parts) * kTiles;  // the CTA's first tile
+    const ChunkItem it = item_of(kGridItem);
+    if (tid == 0 && it.err_count && dev_error) atomicAdd(dev_error, it.err_count);
+    if (it.skip) return;  // uniform over the CTA, before any barrier
   }
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool counter = part == 0 && kvh == 0 && qtile == 0 && tid == 0 && dev_error;
-
-  // ---- the CTA's rows and keys (uniform over the CTA; exits before any barrier)
-  int L = context_lens[seq];
-  if (L < 0 || L > max_context_len) {
-    if (counter) atomicAdd(dev_error, 1);
-    L = L < 0 ? 0 : max_context_len;
-  }
-  const int q0 = q_start[seq];
-  int Tq = q_start[seq + 1] - q0;
-  if (q0 < 0 || Tq < 0 || q0 + Tq > num_q_tokens) {
-    if (counter) atomicAdd(dev_error, 1);
-    return;
-  }
-  if (Tq > min(L, max_query_len)) {
-    if (counter) atomicAdd(dev_error, 1);
-    Tq = min(L, max_query_len);
-  }
-  const int tok_per_tile = kRows / group;
-  const int t0 = qtile * tok_per_tile;  // first query token of the CTA
-  if (t0 >= Tq) return;
-  const int nblk_seq = (L + 15) / 16;
-  const int n_parts = nblk_seq > 0 ? (nblk_seq + part_blocks - 1) / part_blocks : 1;
-  if (part >= n_parts) return;
-  const int key_begin = part * part_blocks * 16;
-  const int t_last = min(t0 + kTiles * tok_per_tile, Tq) - 1;  // last query token of the CTA
-  // keys this CTA can see in this partition: up to the last row's causal limit
-  const int key_end = min(min((part + 1) * part_blocks * 16, L), L - Tq + t_last + 1);
-  const int n_steps = key_end > key_begin ? (key_end - key_begin + kKeys - 1) / kKeys : 0;
-  const int q_head0 = kvh * group;
 
   // ---- set-up: barriers (thread 0), TMEM (warp 0)
   if (tid == 0) {
@@ -207,6 +264,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     mbar_init(o_done, 1);
     mbar_init(mma_drain, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_empty[i], 1 + kSoftmaxWarps);  // the MMA warp, each softmax warp
+    }
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -219,10 +281,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t tmem = *tmem_slot;
   bool failed = false;
 
+  // The k-th item of this CTA, for the MMA and softmax warps (whole warp): its
+  // index into the plan's list x KV heads, kGridItem in grid mode, or -1 when
+  // there is none (or the wait for it gave up: failed is then set).
+  auto take_item = [&](int k) -> int {
+    if (!persistent) return k == 0 ? kGridItem : -1;
+    const int slot = k & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(&item_full[slot], (uint32_t)((k >> 1) & 1)))) {
+      failed = true;
+      return -1;
+    }
+    const int w = *reinterpret_cast<volatile int32_t*>(&item_slot[slot]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[slot]);
+    return w;
+  };
+
   const uint32_t q_s = smem_addr(smem + kQOff);
   auto stage_k = [&](int st) { return smem + kKOff + st * kKBytes; };
   auto stage_v = [&](int st) { return smem + kVOff + st * kVBytes; };
-  const int32_t* bt_row = block_tables + (size_t)seq * bt_stride;
 
   if (warp == kLoadWarp) {
     // ============================ TMA loads =================================
@@ -231,92 +308,121 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // (K, then V) lane 0 posts the expected bytes and lanes 0-15 issue the
     // step's sixteen box copies (8 cache blocks x 2 column chunks) in one
     // instruction. A stage is refilled once the MMAs that read it committed
-    // its "empty" barrier; the loads run up to kStages steps ahead.
-    const int lb_first = key_begin / 16;
-    const int nblk_keys = (key_end - key_begin + 15) / 16;
-    // A table entry outside the pool is skipped (not loaded; the softmax
-    // masks its keys) and counted once: by the KV-head-0 CTA of the last
-    // pair of query tiles, whose causal horizon covers the whole partition.
-    const bool count_bad =
-        dev_error && kvh == 0 && t0 + kTiles * tok_per_tile >= Tq;
-    auto load_window = [&](int w) {
-      const int i = 32 * w + lane;
-      int p = -1;
-      if (i < nblk_keys) {
-        p = __ldg(bt_row + lb_first + i);
-        if (p < 0 || p >= num_blocks) {
-          if (count_bad) atomicAdd(dev_error, 1);
-          p = -1;
-        }
-      }
-      return p;
-    };
-    int win = 0, pid_cur = load_window(0), pid_nxt = load_window(1);
-    auto pid_of = [&](int i) {  // all lanes; i / 32 uniform over the warp
-      const int w = i >> 5;
-      if (w != win && w != win + 1) {  // outside the register window: read the table
-        const int p = i < nblk_keys ? __ldg(bt_row + lb_first + i) : -1;
-        return (p < 0 || p >= num_blocks) ? -1 : p;
-      }
-      const int v = w == win ? pid_cur : pid_nxt;
-      return __shfl_sync(0xffffffffu, v, i & 31);
-    };
-    // K (or V) of step j's eight cache blocks into stage j % kStages; blocks
-    // past the keys or with a bad table entry are not loaded.
-    auto load = [&](int j, bool is_v) {
-      const int st = j % kStages;
-      uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
-      uint8_t* dst = is_v ? stage_v(st) : stage_k(st);
-      const CUtensorMap* map = is_v ? &tm_v : &tm_k;
-      while (((j * kStepBlocks) >> 5) > win) {  // a step's 8 entries share one window
-        ++win;
-        pid_cur = pid_nxt;
-        pid_nxt = load_window(win + 1);
-      }
-      const int b = (lane >> 1) & (kStepBlocks - 1), c = lane & 1;  // lanes 0-15: block, chunk
-      const int pid = pid_of(j * kStepBlocks + b);
-      const bool mine = lane < kStepBlocks * kChunks && pid >= 0;
-      const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, mine)) * 2048u;
-      if (lane == 0) {
-        if (bytes) mbar_arrive_expect_tx(bar, bytes);
-        else mbar_arrive(bar);  // nothing to load: complete the phase empty
-      }
-      __syncwarp();
-      if (mine) tma_load_4d(dst + c * (kKeys * 128) + b * 2048, map, bar, c * 64, 0, kvh, pid);
-    };
+    // its "empty" barrier; the loads run up to kStages steps ahead, across
+    // items. An item's Q follows its first K and V, once the previous item's
+    // last S MMAs are done with the Q tiles.
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity));
     };
-    int nk = 0, nv = 0;  // steps whose K / V loads were issued
-    if (n_steps > 0) {
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        // Both tiles' rows; rows past the q buffer read as zeros (and are
-        // never written out).
-        mbar_arrive_expect_tx(q_full, kTiles * kQBytes);
-#pragma unroll
-        for (int i = 0; i < kTiles; ++i)
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c)
-            tc::tma_load_3d(smem + kQOff + i * kQBytes + c * (kRows * 128), &tm_q, q_full,
-                            c * 64, q_head0, q0 + t0 + i * tok_per_tile);
+    int nk = 0, nv = 0, nq = 0;  // K / V steps and Q loads issued, over all items
+    // plan mode: the next item, fetched by lane 0 and posted in its slot
+    auto fetch_item = [&](int k) {
+      const int slot = k & 1;
+      if (k >= 2 && !wait_all(&item_empty[slot], (uint32_t)(((k >> 1) - 1) & 1))) {
+        failed = true;
+        return -1;
       }
-      for (int j = 0; j < n_steps; ++j) {
-        const uint32_t reuse = (uint32_t)((j / kStages - 1) & 1);
-        if (j >= kStages && !wait_all(&k_empty[j % kStages], reuse)) { failed = true; break; }
-        load(j, false);
+      int w = -1;
+      if (lane == 0) {
+        const int64_t n_work = (int64_t)plan[0] * num_kv_heads;
+        const int64_t c = atomicAdd(&plan[1], 1);
+        w = c < n_work ? (int)c : -1;
+        item_slot[slot] = w;
+        mbar_arrive(&item_full[slot]);  // release: the slot write is visible to its waiters
+      }
+      return __shfl_sync(0xffffffffu, w, 0);
+    };
+    for (int k = 0; !failed; ++k) {
+      const int w = persistent ? fetch_item(k) : (k == 0 ? kGridItem : -1);
+      if (w == -1) break;
+      const ChunkItem it = item_of(w);
+      if (it.skip || it.n_steps == 0) continue;
+      const int32_t* bt_row = block_tables + (size_t)it.seq * bt_stride;
+      const int lb_first = it.key_begin / 16;
+      const int nblk_keys = (it.key_end - it.key_begin + 15) / 16;
+      const int tok_per_tile = kRows / group;
+      // A table entry outside the pool is skipped (not loaded; the softmax
+      // masks its keys) and counted once: by the KV-head-0 item of the last
+      // pair of query tiles, whose causal horizon covers the whole partition.
+      const bool count_bad = dev_error && it.kvh == 0 && it.t0 + kTiles * tok_per_tile >= it.Tq;
+      auto load_window = [&](int wi) {  // entries 32 wi .. 32 wi + 31 of the item's keys
+        const int i = 32 * wi + lane;
+        int p = -1;
+        if (i < nblk_keys) {
+          p = __ldg(bt_row + lb_first + i);
+          if (p < 0 || p >= num_blocks) {
+            if (count_bad) atomicAdd(dev_error, 1);
+            p = -1;
+          }
+        }
+        return p;
+      };
+      int win = 0, pid_cur = load_window(0), pid_nxt = load_window(1);
+      auto pid_of = [&](int i) {  // all lanes; i / 32 uniform over the warp
+        const int wi = i >> 5;
+        if (wi != win && wi != win + 1) {  // outside the register window: read the table
+          const int p = i < nblk_keys ? __ldg(bt_row + lb_first + i) : -1;
+          return (p < 0 || p >= num_blocks) ? -1 : p;
+        }
+        const int v = wi == win ? pid_cur : pid_nxt;
+        return __shfl_sync(0xffffffffu, v, i & 31);
+      };
+      // K (or V) of the item's step j (global step g) into stage g % kStages;
+      // blocks past the keys or with a bad table entry are not loaded.
+      auto load = [&](int j, int g, bool is_v) {
+        const int st = g % kStages;
+        uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
+        uint8_t* dst = is_v ? stage_v(st) : stage_k(st);
+        const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+        while (((j * kStepBlocks) >> 5) > win) {  // a step's 8 entries share one window
+          ++win;
+          pid_cur = pid_nxt;
+          pid_nxt = load_window(win + 1);
+        }
+        const int b = (lane >> 1) & (kStepBlocks - 1), c = lane & 1;  // lanes 0-15: block, chunk
+        const int pid = pid_of(j * kStepBlocks + b);
+        const bool mine = lane < kStepBlocks * kChunks && pid >= 0;
+        const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, mine)) * 2048u;
+        if (lane == 0) {
+          if (bytes) mbar_arrive_expect_tx(bar, bytes);
+          else mbar_arrive(bar);  // nothing to load: complete the phase empty
+        }
+        __syncwarp();
+        if (mine) tma_load_4d(dst + c * (kKeys * 128) + b * 2048, map, bar, c * 64, 0, it.kvh, pid);
+      };
+      for (int j = 0; j < it.n_steps; ++j) {
+        if (nk >= kStages &&
+            !wait_all(&k_empty[nk % kStages], (uint32_t)((nk / kStages - 1) & 1))) { failed = true; break; }
+        load(j, nk, false);
         ++nk;
-        if (j >= kStages && !wait_all(&v_empty[j % kStages], reuse)) { failed = true; break; }
-        load(j, true);
+        if (nv >= kStages &&
+            !wait_all(&v_empty[nv % kStages], (uint32_t)((nv / kStages - 1) & 1))) { failed = true; break; }
+        load(j, nv, true);
         ++nv;
+        if (j == 0) {
+          // Q of both tiles (rows past the q buffer read as zeros and are
+          // never written out), once the previous item's S MMAs are done
+          if (nq > 0 && !wait_all(q_empty, (uint32_t)((nq - 1) & 1))) { failed = true; break; }
+          if (lane == 0) {
+            if (nq == 0) tma_prefetch_desc(&tm_q);
+            mbar_arrive_expect_tx(q_full, kTiles * kQBytes);
+#pragma unroll
+            for (int i = 0; i < kTiles; ++i)
+#pragma unroll
+              for (int c = 0; c < kChunks; ++c)
+                tc::tma_load_3d(smem + kQOff + i * kQBytes + c * (kRows * 128), &tm_q, q_full,
+                                c * 64, it.kvh * group, it.q0 + it.t0 + i * tok_per_tile);
+          }
+          ++nq;
+        }
       }
     }
     if (failed) {
       // Let the copies already issued land (each wait bounded) before the
       // shared memory is released.
-      (void)mbar_wait(q_full, 0);
+      if (nq > 0) (void)mbar_wait(q_full, (uint32_t)((nq - 1) & 1));
       for (int st = 0; st < kStages; ++st) {
-        // the last load issued into stage st is step st + kStages * ((n - 1 - st) / kStages)
+        // the last load issued into stage st is number st + kStages * ((n - 1 - st) / kStages)
         if (nk > st) (void)mbar_wait(&k_full[st], (uint32_t)(((nk - 1 - st) / kStages) & 1));
         if (nv > st) (void)mbar_wait(&v_full[st], (uint32_t)(((nv - 1 - st) / kStages) & 1));
       }
@@ -325,7 +431,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   } else if (warp == kMmaWarp) {
     // ============================== MMAs ====================================
     // One lane issues every tcgen05.mma in the order S_0(j), P.V_1(j-1),
-    // S_1(j), P.V_0(j). Descriptors are built once and offset per MMA.
+    // S_1(j), P.V_0(j) within an item, then the item's last P.V_1; the next
+    // item's S_0(0) follows at once. Descriptors are built once and offset
+    // per MMA; g counts steps over all items (ring stages and barrier phases).
     const bool leader = lane == 0;
     const uint32_t id_s = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kKeys, false, false);
     const uint32_t id_pv = tc::instr_desc_f16(Elem<T>::kBf16, kRows, kD, false, true);
@@ -335,9 +443,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity));
     };
-    // S_i(j) = Q_i K_j^T into tile i's S columns; commit to s_full[i]
-    auto issue_s = [&](int i, int j) {
-      const uint64_t dks = dk + (uint64_t)(((j % kStages) * kKBytes) >> 4);
+    // S_i = Q_i K^T of global step g into tile i's S columns; commit to s_full[i]
+    auto issue_s = [&](int i, int g) {
+      const uint64_t dks = dk + (uint64_t)(((g % kStages) * kKBytes) >> 4);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -349,50 +457,60 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         tc::commit(&s_full[i]);
       }
     };
-    // O_i += P_i(j) V_j, P from TMEM (the first 64 columns of tile i's S)
-    auto issue_pv = [&](int i, int j) {
-      const uint64_t dvs = dv + (uint64_t)(((j % kStages) * kVBytes) >> 4);
+    // O_i += P_i V of global step g, P from TMEM (the first 64 columns of tile
+    // i's S); `first`: the item's first step (O starts from zero)
+    auto issue_pv = [&](int i, int g, bool first) {
+      const uint64_t dvs = dv + (uint64_t)(((g % kStages) * kVBytes) >> 4);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           const uint64_t b = dvs + (uint64_t)((kk * 2048) >> 4);
           tc::mma_f16_tmem_a(tmem + (uint32_t)(i * kTileCols) + kOCol,
                              tmem + (uint32_t)(i * kTileCols) + (uint32_t)(kk * 8), b, id_pv,
-                             j > 0 || kk > 0);
+                             !first || kk > 0);
         }
       }
     };
-    if (n_steps > 0 && !wait_all(q_full, 0)) failed = true;
-    for (int j = 0; j < n_steps && !failed; ++j) {
-      const int st = j % kStages;
-      if (!wait_all(&k_full[st], (uint32_t)((j / kStages) & 1))) { failed = true; break; }
-      tc::fence_after_sync();
-      issue_s(0, j);
-      if (j > 0) {  // P.V_1(j-1): V(j-1) landed (awaited before P.V_0(j-1))
-        if (!wait_all(&p_ready[1], (uint32_t)((j - 1) & 1))) { failed = true; break; }
+    int g0 = 0, nq = 0;  // steps and Q tiles consumed by earlier items
+    for (int k = 0; !failed; ++k) {
+      const int w = take_item(k);
+      if (w == -1) break;
+      const ChunkItem it = item_of(w);
+      if (it.skip || it.n_steps == 0) continue;
+      const int n = it.n_steps;
+      if (!wait_all(q_full, (uint32_t)(nq & 1))) { failed = true; break; }
+      ++nq;
+      for (int j = 0; j < n; ++j) {
+        const int g = g0 + j, st = g % kStages;
+        if (!wait_all(&k_full[st], (uint32_t)((g / kStages) & 1))) { failed = true; break; }
         tc::fence_after_sync();
-        issue_pv(1, j - 1);
-        if (leader) tc::commit(&v_empty[(j - 1) % kStages]);
-      }
-      issue_s(1, j);
-      if (leader) tc::commit(&k_empty[st]);  // K stage st free once S_0(j), S_1(j) completed
-      if (!wait_all(&v_full[st], (uint32_t)((j / kStages) & 1))) { failed = true; break; }
-      if (!wait_all(&p_ready[0], (uint32_t)(j & 1))) { failed = true; break; }
-      tc::fence_after_sync();
-      issue_pv(0, j);
-    }
-    if (!failed && n_steps > 0) {
-      const int jl = n_steps - 1;
-      if (!wait_all(&p_ready[1], (uint32_t)(jl & 1))) {
-        failed = true;
-      } else {
-        tc::fence_after_sync();
-        issue_pv(1, jl);
-        if (leader) {
-          tc::commit(&v_empty[jl % kStages]);
-          tc::commit(o_done);  // both tiles' O are final once this completes
+        issue_s(0, g);
+        if (j > 0) {  // P.V_1(j-1): V(j-1) landed (awaited before P.V_0(j-1))
+          if (!wait_all(&p_ready[1], (uint32_t)((g - 1) & 1))) { failed = true; break; }
+          tc::fence_after_sync();
+          issue_pv(1, g - 1, j == 1);
+          if (leader) tc::commit(&v_empty[(g - 1) % kStages]);
         }
+        issue_s(1, g);
+        if (leader) {
+          tc::commit(&k_empty[st]);  // K stage st free once S_0, S_1 of step g completed
+          if (j == n - 1) tc::commit(q_empty);  // the item's last S MMAs: Q reusable after them
+        }
+        if (!wait_all(&v_full[st], (uint32_t)((g / kStages) & 1))) { failed = true; break; }
+        if (!wait_all(&p_ready[0], (uint32_t)(g & 1))) { failed = true; break; }
+        tc::fence_after_sync();
+        issue_pv(0, g, j == 0);
       }
+      if (failed) break;
+      const int gl = g0 + n - 1;
+      if (!wait_all(&p_ready[1], (uint32_t)(gl & 1))) { failed = true; break; }
+      tc::fence_after_sync();
+      issue_pv(1, gl, n == 1);
+      if (leader) {
+        tc::commit(&v_empty[gl % kStages]);
+        tc::commit(o_done);  // both tiles' O of the item are final once this completes
+      }
+      g0 += n;
     }
     if (failed) {
       // The MMAs already issued finish (bounded wait) before TMEM is released:
@@ -408,164 +526,179 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int r = tid & (kRows - 1);                     // tile row = TMEM lane
     const uint32_t lane_addr =
         tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(tile * kTileCols);
-    const int tt0 = t0 + tile * tok_per_tile;            // first query token of the tile
-    const int t = tt0 + r / group, h = r % group;        // query token in the chunk, head
-    const bool row_ok = t < Tq;
-    const int lim = L - Tq + (row_ok ? t : 0);           // last key this row may see
-    float m = -INFINITY, l = 0.f;                        // reference maximum (log2 units)
-    // keys every row of the tile may see: up to the first row's causal limit
-    const int key_all = min(key_end, L - Tq + tt0 + 1);
-    // Validity of the table entries of a step (a bit per cache block), loaded
-    // one step ahead so the table reads never wait in the loop.
-    auto bad_blocks = [&](int j) {
-      int mask = 0;
-      const int lb0 = (key_begin + j * kKeys) / 16;
+    int g = 0, no = 0;  // steps (over all items) and O results consumed so far
+    for (int k = 0; !failed; ++k) {
+      const int w = take_item(k);
+      if (w == -1) break;
+      const ChunkItem it = item_of(w);
+      if (persistent && tid == 0 && it.err_count && dev_error) atomicAdd(dev_error, it.err_count);
+      if (it.skip) continue;
+      const int key_begin = it.key_begin, key_end = it.key_end, seq = it.seq;
+      const int L = it.L, Tq = it.Tq;
+      const int tok_per_tile = kRows / group;
+      const int tt0 = it.t0 + tile * tok_per_tile;       // first query token of the tile
+      const int t = tt0 + r / group;                     // query token in the chunk
+      const bool row_ok = t < Tq;
+      // the row's output: out row, and the partition (-1: one partition, direct)
+      const size_t orow = (size_t)(it.q0 + t) * num_q_heads + it.kvh * group + r % group;
+      const int opart = it.n_parts == 1 ? -1 : it.part;
+      const int lim = L - Tq + (row_ok ? t : 0);         // last key this row may see
+      float m = -INFINITY, l = 0.f;                      // reference maximum (log2 units)
+      // keys every row of the tile may see: up to the first row's causal limit
+      const int key_all = min(key_end, L - Tq + tt0 + 1);
+      // Validity of the table entries of the step at key kb0 (a bit per cache
+      // block), loaded one step ahead so the table reads never wait in the loop.
+      auto bad_blocks = [&](int kb0) {
+        const int32_t* bt_row = block_tables + (size_t)seq * bt_stride;
+        int mask = 0;
 #pragma unroll
-      for (int b = 0; b < kStepBlocks; ++b) {
-        const int lb = lb0 + b;
-        if (lb * 16 < key_end) {
-          const int p = __ldg(bt_row + lb);
-          if (p < 0 || p >= num_blocks) mask |= 1 << b;
-        }
-      }
-      return mask;
-    };
-    int bad_next = n_steps > 0 ? bad_blocks(0) : 0;
-    for (int j = 0; j < n_steps; ++j) {
-      const int st = j % kStages;
-      const int kb = key_begin + j * kKeys;
-      const int bad_mask = bad_next;
-      if (j + 1 < n_steps) bad_next = bad_blocks(j + 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], (uint32_t)(j & 1)))) { failed = true; break; }
-      tc::fence_after_sync();
-      float s[kKeys];
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        float v[32];
-        tc::tmem_ld32(lane_addr + (uint32_t)(c * 32), v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = v[i];
-      }
-      tc::tmem_wait_ld();
-      // Logits in log2 units are s * scale_log2. Steps wholly inside the
-      // tile's causal horizon need no mask (scale folded into the exp's FMA);
-      // otherwise scale first and give masked keys -inf.
-      const bool need_mask = kb + kKeys > key_all || bad_mask != 0;
-      float mx, cc;
-      if (need_mask) {
-        mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < kKeys; ++i) {
-          const int kp = kb + i;
-          const bool ok = kp < key_end && kp <= lim && !((bad_mask >> (i >> 4)) & 1);
-          s[i] = ok ? s[i] * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[i]);
-        }
-        cc = 1.f;
-      } else {
-        // the largest logit is the largest raw score (the smallest, for a
-        // negative scale); four independent chains of three-input max
-        static_assert(kKeys % 8 == 4 || kKeys % 8 == 0, "reduction layout");
-        float e0 = s[0], e1 = s[1], e2 = s[2], e3 = s[3];
-        if (scale_log2 >= 0.f) {
-#pragma unroll
-          for (int i = 4; i + 8 <= kKeys; i += 8) {
-            e0 = max3(e0, s[i], s[i + 1]);
-            e1 = max3(e1, s[i + 2], s[i + 3]);
-            e2 = max3(e2, s[i + 4], s[i + 5]);
-            e3 = max3(e3, s[i + 6], s[i + 7]);
+        for (int b = 0; b < kStepBlocks; ++b) {
+          const int lb = kb0 / 16 + b;
+          if (lb * 16 < key_end) {
+            const int p = __ldg(bt_row + lb);
+            if (p < 0 || p >= num_blocks) mask |= 1 << b;
           }
-          e0 = max3(e0, s[kKeys - 4], s[kKeys - 3]);
-          e1 = max3(e1, s[kKeys - 2], s[kKeys - 1]);
-          mx = max3(e0, e1, fmaxf(e2, e3)) * scale_log2;
+        }
+        return mask;
+      };
+      int bad_next = key_begin < key_end ? bad_blocks(key_begin) : 0;
+      // one step per 128 keys; g counts steps over all items
+      for (int kb = key_begin; kb < key_end; kb += kKeys, ++g) {
+        const int st = g % kStages;
+        const int bad_mask = bad_next;
+        if (kb + kKeys < key_end) bad_next = bad_blocks(kb + kKeys);
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], (uint32_t)(g & 1)))) { failed = true; break; }
+        tc::fence_after_sync();
+        float s[kKeys];
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(lane_addr + (uint32_t)(c * 32), v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = v[i];
+        }
+        tc::tmem_wait_ld();
+        // Logits in log2 units are s * scale_log2. Steps wholly inside the
+        // tile's causal horizon need no mask (scale folded into the exp's FMA);
+        // otherwise scale first and give masked keys -inf.
+        const bool need_mask = kb + kKeys > key_all || bad_mask != 0;
+        float mx, cc;
+        if (need_mask) {
+          mx = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < kKeys; ++i) {
+            const int kp = kb + i;
+            const bool ok = kp < key_end && kp <= lim && !((bad_mask >> (i >> 4)) & 1);
+            s[i] = ok ? s[i] * scale_log2 : -INFINITY;
+            mx = fmaxf(mx, s[i]);
+          }
+          cc = 1.f;
         } else {
+          // the largest logit is the largest raw score (the smallest, for a
+          // negative scale); four independent chains of three-input max
+          static_assert(kKeys % 8 == 4 || kKeys % 8 == 0, "reduction layout");
+          float e0 = s[0], e1 = s[1], e2 = s[2], e3 = s[3];
+          if (scale_log2 >= 0.f) {
 #pragma unroll
-          for (int i = 4; i + 8 <= kKeys; i += 8) {
-            e0 = min3(e0, s[i], s[i + 1]);
-            e1 = min3(e1, s[i + 2], s[i + 3]);
-            e2 = min3(e2, s[i + 4], s[i + 5]);
-            e3 = min3(e3, s[i + 6], s[i + 7]);
-          }
-          e0 = min3(e0, s[kKeys - 4], s[kKeys - 3]);
-          e1 = min3(e1, s[kKeys - 2], s[kKeys - 1]);
-          mx = min3(e0, e1, fminf(e2, e3)) * scale_log2;
-        }
-        cc = scale_log2;
-      }
-      float alpha = 1.f;
-      if (mx > m + kRescaleLog2 || m == -INFINITY) {
-        const float m_new = fmaxf(m, mx);
-        alpha = m == -INFINITY ? 0.f : fast_exp2(m - m_new);
-        m = m_new;
-      }
-      const float m_use = m == -INFINITY ? 0.f : m;
-      // P_j row r: 128 bf16 = 64 columns over the S columns already read
-      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;  // four chains of row-sum adds
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(s[32 * c + 2 * i], cc, -m_use));
-          const float p1 = fast_exp2(fmaf(s[32 * c + 2 * i + 1], cc, -m_use));
-          if (i & 1) {
-            sa1 += p0;
-            sb1 += p1;
+            for (int i = 4; i + 8 <= kKeys; i += 8) {
+              e0 = max3(e0, s[i], s[i + 1]);
+              e1 = max3(e1, s[i + 2], s[i + 3]);
+              e2 = max3(e2, s[i + 4], s[i + 5]);
+              e3 = max3(e3, s[i + 6], s[i + 7]);
+            }
+            e0 = max3(e0, s[kKeys - 4], s[kKeys - 3]);
+            e1 = max3(e1, s[kKeys - 2], s[kKeys - 1]);
+            mx = max3(e0, e1, fmaxf(e2, e3)) * scale_log2;
           } else {
-            sa0 += p0;
-            sb0 += p1;
+#pragma unroll
+            for (int i = 4; i + 8 <= kKeys; i += 8) {
+              e0 = min3(e0, s[i], s[i + 1]);
+              e1 = min3(e1, s[i + 2], s[i + 3]);
+              e2 = min3(e2, s[i + 4], s[i + 5]);
+              e3 = min3(e3, s[i + 6], s[i + 7]);
+            }
+            e0 = min3(e0, s[kKeys - 4], s[kKeys - 3]);
+            e1 = min3(e1, s[kKeys - 2], s[kKeys - 1]);
+            mx = min3(e0, e1, fminf(e2, e3)) * scale_log2;
           }
-          pk[i] = E::pack(p0, p1);
+          cc = scale_log2;
         }
-        tc::tmem_st16u(lane_addr + (uint32_t)(c * 16), pk);
-      }
-      l = l * alpha + ((sa0 + sa1) + (sb0 + sb1));
-      // rescale O when a row's reference maximum moved (warp-uniform
-      // decision); P.V_tile(j-1) has completed (covered by s_full's commit),
-      // P.V_tile(j) waits for this warp's p_ready arrival
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        float alpha = 1.f;
+        if (mx > m + kRescaleLog2 || m == -INFINITY) {
+          const float m_new = fmaxf(m, mx);
+          alpha = m == -INFINITY ? 0.f : fast_exp2(m - m_new);
+          m = m_new;
+        }
+        const float m_use = m == -INFINITY ? 0.f : m;
+        // P_j row r: 128 bf16 = 64 columns over the S columns already read
+        float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;  // four chains of row-sum adds
 #pragma unroll
-        for (int c = 0; c < kD / 32; ++c) {
-          float o[32];
-          tc::tmem_ld32(lane_addr + kOCol + c * 32, o);
-          tc::tmem_wait_ld();
+        for (int c = 0; c < kKeys / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tc::tmem_st32(lane_addr + kOCol + c * 32, o);
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(s[32 * c + 2 * i], cc, -m_use));
+            const float p1 = fast_exp2(fmaf(s[32 * c + 2 * i + 1], cc, -m_use));
+            if (i & 1) {
+              sa1 += p0;
+              sb1 += p1;
+            } else {
+              sa0 += p0;
+              sb0 += p1;
+            }
+            pk[i] = E::pack(p0, p1);
+          }
+          tc::tmem_st16u(lane_addr + (uint32_t)(c * 16), pk);
         }
-      }
-      tc::tmem_wait_st();
-      // V rows of keys past the context or of bad blocks become zero (once V_j
-      // landed); tile 0 does it, before its p_ready, which the MMA warp awaits
-      // before either tile's P.V(j).
-      if (tile == 0 && (kb + kKeys > key_end || bad_mask)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (uint32_t)((j / kStages) & 1)))) { failed = true; break; }
-        uint8_t* v = stage_v(st);
-        for (int i = r; i < kKeys * kChunks * 8; i += kRows) {
-          const int c = i / (kKeys * 8), rem = i % (kKeys * 8);
-          const int key = rem / 8;
-          if (kb + key >= key_end || ((bad_mask >> (key >> 4)) & 1))
-            *reinterpret_cast<uint4*>(v + c * (kKeys * 128) + key * 128 + (rem % 8) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
+        l = l * alpha + ((sa0 + sa1) + (sb0 + sb1));
+        // rescale O when a row's reference maximum moved (warp-uniform
+        // decision; not at an item's first step, where P.V starts O afresh);
+        // the previous step's P.V of this tile has completed (covered by
+        // s_full's commit), this step's waits for this warp's p_ready arrival
+        if (kb > key_begin && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c) {
+            float o[32];
+            tc::tmem_ld32(lane_addr + kOCol + c * 32, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tc::tmem_st32(lane_addr + kOCol + c * 32, o);
+          }
         }
-        fence_proxy_async_smem();  // zeroed V rows -> visible to the tensor core
+        tc::tmem_wait_st();
+        // V rows of keys past the context or of bad blocks become zero (once V
+        // landed); tile 0 does it, before its p_ready, which the MMA warp awaits
+        // before either tile's P.V of the step.
+        if (tile == 0 && (kb + kKeys > key_end || bad_mask)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&v_full[st], (uint32_t)((g / kStages) & 1)))) { failed = true; break; }
+          uint8_t* v = stage_v(st);
+          for (int i = r; i < kKeys * kChunks * 8; i += kRows) {
+            const int c = i / (kKeys * 8), rem = i % (kKeys * 8);
+            const int key = rem / 8;
+            if (kb + key >= key_end || ((bad_mask >> (key >> 4)) & 1))
+              *reinterpret_cast<uint4*>(v + c * (kKeys * 128) + key * 128 + (rem % 8) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();  // zeroed V rows -> visible to the tensor core
+        }
+        tc::fence_before_sync();
+        mbar_arrive(&p_ready[tile]);
       }
-      tc::fence_before_sync();
-      mbar_arrive(&p_ready[tile]);
-    }
-    // ---- epilogue: O / l  ->  out (one partition) or fp32 partials
-    if (!failed && n_steps > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done, 0))) failed = true;
-    if (failed) {
-      if (lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
-    } else {
-      tc::fence_after_sync();
-      const bool direct = n_parts == 1;
-      const size_t orow = (size_t)(q0 + t) * num_q_heads + q_head0 + h;
+      if (failed) break;
+      // ---- the item's epilogue: O / l  ->  out (one partition) or fp32 partials
+      const bool any = key_end > key_begin;  // the item had steps (and MMAs)
+      if (any) {
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)(no & 1)))) { failed = true; break; }
+        ++no;
+        tc::fence_after_sync();
+      }
+      const bool direct = opart < 0;
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         float o[32];
-        if (n_steps > 0) {
+        if (any) {
           tc::tmem_ld32(lane_addr + kOCol + c * 32, o);
           tc::tmem_wait_ld();
         } else {
@@ -582,7 +715,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                                   E::pack(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
                                   E::pack(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
           } else {
-            float4* dst = reinterpret_cast<float4*>(part_o + (orow * max_parts + part) * kD + c * 32);
+            float4* dst = reinterpret_cast<float4*>(part_o + (orow * max_parts + opart) * kD + c * 32);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
@@ -591,8 +724,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
       }
       if (row_ok && !direct)
-        part_lse[orow * max_parts + part] = l > 0.f ? m + log2f(l) : -INFINITY;
+        part_lse[orow * max_parts + opart] = l > 0.f ? m + log2f(l) : -INFINITY;
     }
+    if (failed && lane == 0 && dev_error) atomicAdd(dev_error, PA_DEV_ERR_TIMEOUT);
   }
 
   // ---- teardown: every thread done with TMEM, then warp 0 frees it
@@ -679,7 +813,10 @@ __global__ void __launch_bounds__(kPlanThreads)
   __syncthreads();
   const int incl = x + (warp > 0 ? warp_sum[warp - 1] : 0);
   cursor[b] = incl - v;
-  if (tid == kPlanThreads - 1) plan[0] = incl;
+  if (tid == kPlanThreads - 1) {
+    plan[0] = incl;  // items listed
+    plan[1] = 0;     // work counter of the persistent chunk kernel
+  }
   __syncthreads();
   for (int s = tid; s < num_seqs; s += kPlanThreads)
     visit(s, [&](int local, int steps) {
@@ -729,18 +866,25 @@ cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q,
           a.max_parts, a.dev_error, nullptr, nullptr, a.num_kv_heads);
       return cudaGetLastError();
     }
-    // Longest first: the plan kernel lists the items, the chunk kernel (a
-    // programmatic dependent: resident while the plan runs, reading nothing
-    // before griddepcontrol.wait) takes them in that order.
+    // Longest first: the plan kernel lists the items and zeroes the work
+    // counter; the chunk kernel (a programmatic dependent: resident while the
+    // plan runs, reading nothing before griddepcontrol.wait) runs one CTA per
+    // SM, each taking the next item of the list from the counter when it is
+    // ready for one.
     const int64_t n_max = prefill_tc_max_items(a.num_seqs, a.max_query_len, a.group,
                                                a.max_parts) * a.num_kv_heads;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t ctas = n_max < (int64_t)sms ? n_max : (int64_t)sms;  // one CTA per SM fits
     chunk_plan_kernel<<<1, kPlanThreads, 0, stream>>>(
         a.context_lens, a.q_start, a.num_seqs, a.num_q_tokens, a.max_query_len,
         a.max_context_len, a.group, a.part_blocks, a.max_parts, a.chunk_items, a.chunk_plan);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)n_max);
+    cfg.gridDim = dim3((unsigned)(ctas > 0 ? ctas : 1));
     cfg.blockDim = dim3(kThreadsTc);
     cfg.dynamicSmemBytes = kSmemAlloc;
     cfg.stream = stream;
@@ -755,7 +899,7 @@ cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q,
                               a.group, a.num_blocks, a.max_context_len, a.scale_log2,
                               a.part_blocks, a.max_parts, a.dev_error,
                               static_cast<const uint2*>(a.chunk_items),
-                              static_cast<const int32_t*>(a.chunk_plan), a.num_kv_heads);
+                              a.chunk_plan, a.num_kv_heads);
   };
   return a.bf16 ? run((__nv_bfloat16*)nullptr) : run((__half*)nullptr);
 }

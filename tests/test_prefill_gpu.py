@@ -185,3 +185,23 @@ def test_tensor_core_groups_and_fp16(Hq, Hkv, dtype, P):
     w = W.chunk_workload("tcg", [700, 1500, 260], [120, 64, 260], num_q_heads=Hq,
                          num_kv_heads=Hkv, head_dim=128, dtype=dtype, seed=Hq * 3 + Hkv + P)
     _check(w, P)
+
+
+@pytest.mark.parametrize("P", [0, 128])
+def test_longest_first_chunk_path_over_many_items(P):
+    """With the chunk workspace the tcgen05 path runs one CTA per SM, each
+    taking (tile pair, partition, KV head) items of the longest-first list from
+    a work counter until none is left, its TMEM and barriers carried from item
+    to item. 476 items (no split) and 1,542 (128-token partitions) over 148
+    SMs: ragged chunks, empty chunks, an empty context, and items whose
+    partition lies past their rows' causal limit (no keys: zero partials). The
+    result is the grid order's bit for bit and the oracle's within tolerance."""
+    rng = np.random.default_rng(77 + P)
+    S = 220
+    lens = rng.integers(0, 700, size=S)
+    tq = np.minimum(lens, rng.integers(0, 72, size=S))
+    tq[::17] = 0
+    lens[5], tq[5] = 0, 0
+    w = W.chunk_workload("many", lens, tq, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                         dtype="bf16", seed=78 + P)
+    _check(w, P)
