@@ -844,8 +844,9 @@ def workload_record(name, res, agg, args, world, ceiling) -> dict:
                      else "write_kv + attention") + " (partitions + LSE reduce when split)",
             "scheduler": ("persistent: plan kernel + work-queue grid of SMs x resident CTAs"
                           if res["persistent"] else
-                          "longest first: plan kernel + one CTA per (query-tile pair, partition, "
-                          "KV head, sequence) in descending key count" if res.get("tc_path") else
+                          "longest first, persistent: plan kernel (items in descending key "
+                          "count) + one CTA per SM taking (query-tile pair, partition, KV head, "
+                          "sequence) items from a work counter" if res.get("tc_path") else
                           "grid: one CTA per (partition, KV head, sequence)"),
             "accumulate": "fp32",
             "l2": l2_note(w),
