@@ -394,7 +394,7 @@ int32_t pa_bm_refcount(const pa_block_manager* bm, int32_t block);
  * multiple of 16) once with every SM and discards them:
  *   method 0: 128-bit loads that bypass L1, eight in flight per thread,
  *             every resident thread sweeping the buffer;
- *   method 1: bulk asynchronous copies (cp.async.bulk, 16 KiB, no multicast)
+ *   method 1: bulk asynchronous copies (cp.async.bulk, 16 KiB, into the issuing CTA)
  *             into a shared-memory ring per CTA -- the engine the decode
  *             kernels read their tiles with;
  *   method 2: the paged decode's access pattern without its arithmetic: the

@@ -105,7 +105,7 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 
 // ---------------------------------------------------------------- TMA
 // Tiled 4-D tensor load into this CTA's shared memory, completion counted on
-// `bar` in bytes. No multicast.
+// `bar` in bytes; this CTA's own destination only.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(

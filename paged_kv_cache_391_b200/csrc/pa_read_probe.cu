@@ -7,7 +7,7 @@
 //   method 0: 128-bit loads that bypass L1, eight in flight per thread, a
 //             grid-stride sweep by every resident thread; the words are
 //             XOR-folded so the loads cannot be dropped;
-//   method 1: bulk asynchronous copies (cp.async.bulk, no multicast) of 16 KiB
+//   method 1: bulk asynchronous copies (cp.async.bulk, into this CTA only) of 16 KiB
 //             chunks into a 6-stage shared-memory ring per CTA, mbarrier
 //             tracked -- the same engine the decode kernels read tiles with.
 //   method 2: scattered 4 KiB tiles by 2 KiB TMA tensor boxes, in the decode

@@ -166,7 +166,7 @@ __device__ __forceinline__ void commit(uint64_t* bar) {
       : "memory");
 }
 
-// Tiled 3-D TMA load (no multicast).
+// Tiled 3-D TMA load into this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
   asm volatile(
