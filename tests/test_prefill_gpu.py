@@ -205,3 +205,33 @@ def test_longest_first_chunk_path_over_many_items(P):
     w = W.chunk_workload("many", lens, tq, num_q_heads=8, num_kv_heads=2, head_dim=128,
                          dtype="bf16", seed=78 + P)
     _check(w, P)
+
+
+def test_argument_errors_on_the_tensor_core_path_counted_once_in_both_orders():
+    """Query ranges outside the q rows on the tcgen05 path: each bad sequence
+    is counted exactly once (by its first item) and skipped, whether one CTA
+    runs one item (grid order) or persistent CTAs take the items from the
+    longest-first list; the good sequence's rows are the oracle's."""
+    w = W.chunk_workload("badtc", [300, 400, 500], [40, 50, 60], num_q_heads=8, num_kv_heads=2,
+                         head_dim=128, dtype="bf16", seed=12)
+    d = DeviceStep(w)
+    d.cache_ops()
+    qs = torch.from_numpy(w.q_start).cuda()
+    qs[2] = 10_000          # sequences 1 and 2 now run past the 150 q rows
+    kc, vc = oracle_caches_after_step(w)
+    ref = oracle.prefill_chunk(w.q, w.q_start, kc, vc, w.block_tables, w.context_lens, w.scale,
+                               w.dtype)
+    for ordered in (False, True):
+        ws = (pa.alloc_chunk_workspace(int(w.q.shape[0]), w.num_seqs, w.num_q_heads,
+                                       w.group_size, 128, 60, w.max_context_len, d.P, "cuda")
+              if ordered else d.ws)
+        d.err.zero_()
+        out = torch.full_like(d.out, 5.0)
+        pa.prefill_chunk(out, d.q, qs, d.k_cache, d.v_cache, d.bt, d.cl, scale=w.scale,
+                         max_query_len=60, max_context_len=w.max_context_len,
+                         partition_tokens=d.P, workspace=ws, dev_error=d.err)
+        torch.cuda.synchronize()
+        assert int(d.err.item()) == 2, ordered
+        o = to_f64(out)
+        assert_decode_close(o[:40], ref[:40], f"good sequence, ordered={ordered}")
+        assert (o[40:] == 5.0).all()
