@@ -235,3 +235,23 @@ def test_argument_errors_on_the_tensor_core_path_counted_once_in_both_orders():
         o = to_f64(out)
         assert_decode_close(o[:40], ref[:40], f"good sequence, ordered={ordered}")
         assert (o[40:] == 5.0).all()
+
+
+def test_tensor_core_output_needs_only_16_byte_alignment():
+    """The call asks only for a 16-byte aligned `out`: on the tcgen05 path an
+    output view 16 bytes into a buffer (not 32-byte aligned) gets the aligned
+    output's bits, in both orders, and nothing is written before the view."""
+    w = W.chunk_workload("align", [700, 1500], [120, 64], num_q_heads=8, num_kv_heads=2,
+                         head_dim=128, dtype="bf16", seed=91)
+    d = DeviceStep(w, 0)
+    d.cache_ops()
+    for ordered in (False, True):
+        a = d.prefill(torch.full_like(d.out, float("nan")), ordered=ordered)
+        big = torch.full((d.out.numel() + 8,), float("nan"), dtype=d.out.dtype, device="cuda")
+        b = big[8:].view(d.out.shape)
+        assert a.data_ptr() % 32 == 0 and b.data_ptr() % 32 == 16
+        d.prefill(b, ordered=ordered)
+        torch.cuda.synchronize()
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), ordered
+        assert torch.isnan(big[:8].float()).all()     # nothing written before the view
+    assert int(d.err.item()) == 0
