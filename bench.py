@@ -8,7 +8,7 @@ log-sum-exp reduce when a context spans several partitions), all through
 libpa's C ABI on the current CUDA stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha|gqa|shared_prefix|long|...]
-                  [--scheduler grid|persistent]
+                  [--scheduler grid|persistent|shared]
   python bench.py --impl reference ...   # the fp64 CPU oracle, timed on the host cores
 
 Multi-GPU (launched by torch.distributed.run): every rank runs its own
@@ -73,9 +73,11 @@ def parse():
                     help="step: the decode step (default); swap: preemption swap-out/in; "
                          "blockmgr: host block-manager throughput (no GPU)")
     ap.add_argument("--partition-tokens", type=int, default=None)
-    ap.add_argument("--scheduler", default="grid", choices=["grid", "persistent"],
+    ap.add_argument("--scheduler", default="grid", choices=["grid", "persistent", "shared"],
                     help="decode schedule: grid = pa_decode (one CTA per partition); "
-                         "persistent = pa_decode_persistent (plan + work queue)")
+                         "persistent = pa_decode_persistent (plan + work queue); shared = "
+                         "pa_decode_shared_prefix for the shared_prefix workload (the shared "
+                         "partitions as one tcgen05 contraction over all sequences)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--op-seconds", type=float, default=0.6,
                     help="target GPU time of the write_kv and copy_blocks timing loops")
@@ -447,6 +449,9 @@ def run_gpu(args, name, rank, world, device, probe_buf=None, e2e_on=True):
     P = w.partition_tokens
     n_q = int(w.q.shape[0])
     persistent = args.scheduler == "persistent" and w.q_start is None
+    shared_tokens = (int(w.notes["shared_blocks"]) * 16
+                     if args.scheduler == "shared" and w.q_start is None
+                     and "shared_blocks" in w.notes else 0)
     max_q0 = int(np.diff(w.q_start).max()) if w.q_start is not None else 1
     tc_path = w.q_start is not None and w.head_dim == 128 and max_q0 * w.group_size >= 64
     if w.q_start is not None:   # room for the chunk path's longest-first plan
@@ -461,7 +466,8 @@ def run_gpu(args, name, rank, world, device, probe_buf=None, e2e_on=True):
     max_q = int(np.diff(w.q_start).max()) if w.q_start is not None else 1
     max_parts = 1 if (P == 0 or max_ctx <= P) else -(-max_ctx // P)
     launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + \
-        1 + (1 if max_parts > 1 else 0) + (1 if persistent else 0) + (1 if tc_path else 0)
+        1 + (1 if max_parts > 1 else 0) + (1 if persistent else 0) + (1 if tc_path else 0) + \
+        (1 if shared_tokens else 0)
     copy_pairs_t, copy_what = timing_copy_pairs(w)
     copy_pairs_dev = torch.from_numpy(copy_pairs_t).to(device)
 
@@ -483,7 +489,7 @@ def run_gpu(args, name, rank, world, device, probe_buf=None, e2e_on=True):
         else:
             pa.decode(o, x["q"], k_cache, v_cache, x["bt"], x["cl"], scale=w.scale,
                       max_context_len=max_ctx, partition_tokens=P, workspace=ws, dev_error=err,
-                      stream=stream, persistent=persistent)
+                      stream=stream, persistent=persistent, shared_prefix_tokens=shared_tokens)
 
     def step(x, o):
         copies(x)
@@ -604,7 +610,7 @@ def run_gpu(args, name, rank, world, device, probe_buf=None, e2e_on=True):
             "write_ms": write_ms, "copy_ms": copy_ms, "copy_pairs": int(len(copy_pairs_t)),
             "copy_what": copy_what, "short_reps": short_reps, "rounds": rounds,
             "errors": errors, "e2e": e2e, "launches": launches_per_step,
-            "persistent": persistent, "tc_path": tc_path}
+            "persistent": persistent, "tc_path": tc_path, "shared_tokens": shared_tokens}
 
 
 def l2_note(w) -> str:
@@ -763,6 +769,10 @@ def kernel_name(w, args) -> str:
     if args.scheduler == "persistent":
         return ("pa_decode_persistent (decode_plan_kernel + decode_persistent_kernel + "
                 "lse_reduce_kernel)")
+    if args.scheduler == "shared" and "shared_blocks" in w.notes:
+        return ("pa_decode_shared_prefix (prefill_tc_kernel over the shared partitions of all "
+                "sequences on tcgen05 + decode_partition_kernel over the rest + "
+                "lse_reduce_kernel)")
     return "pa_decode (decode_partition_kernel + lse_reduce_kernel)"
 
 
@@ -844,6 +854,9 @@ def workload_record(name, res, agg, args, world, ceiling) -> dict:
                      else "write_kv + attention") + " (partitions + LSE reduce when split)",
             "scheduler": ("persistent: plan kernel + work-queue grid of SMs x resident CTAs"
                           if res["persistent"] else
+                          f"shared prefix: {res['shared_tokens']} shared tokens, their whole "
+                          "partitions as one tcgen05 contraction over all sequences, the rest "
+                          "as decode partitions" if res.get("shared_tokens") else
                           "longest first, persistent: plan kernel (items in descending key "
                           "count) + one CTA per SM taking (query-tile pair, partition, KV head, "
                           "sequence) items from a work counter" if res.get("tc_path") else

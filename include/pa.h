@@ -180,6 +180,44 @@ pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
                                pa_dtype dtype, void* stream);
 
 /*
+ * pa_decode for a batch whose sequences all begin with the same
+ * shared_prefix_tokens tokens in the same physical blocks: the pages' many
+ * users of one prompt, whose copy-on-write forks share every full prefix
+ * block ("PagedAttention" guide, "KV Cache Sharing (Copy-on-Write)"). Same
+ * arguments and result as pa_decode (within the same tolerance of the exact
+ * attention; not bitwise equal to it). The whole partitions inside the shared
+ * prefix, if there are at least two and they are not all of the longest
+ * context's, are computed once for all sequences: every sequence's query
+ * rows against the prefix keys of sequence 0's table, a dense contraction on
+ * the tcgen05 tensor cores (the chunk kernel, without a causal mask), written
+ * as the decode's fp32 partials; the decode kernel then covers the partitions
+ * after them and the log-sum-exp reduce merges both. Needs head_dim 128, a
+ * power-of-two group_size, num_seqs * group_size >= 64 and partition_tokens a
+ * multiple of 128; otherwise (or when the prefix spans fewer than two whole
+ * partitions) it runs pa_decode.
+ *   shared_prefix_tokens  host, 0 <= shared_prefix_tokens <= max_context_len:
+ *                         tokens at the start of every sequence held in the
+ *                         same blocks as sequence 0's (its first
+ *                         shared_prefix_tokens / 16 table entries, each
+ *                         sequence's context at least that long). A sequence
+ *                         that breaks this over the partitions taken as shared
+ *                         is counted once in dev_error, and its output row is
+ *                         not its attention.
+ *   workspace             >= pa_decode_workspace_size(...) bytes, as pa_decode.
+ * Errors: as pa_decode; PA_ERR_INVALID_ARG also for shared_prefix_tokens
+ * outside [0, max_context_len].
+ */
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  int32_t block_table_stride, const int32_t* context_lens,
+                                  int32_t num_seqs, int32_t num_q_heads, int32_t group_size,
+                                  int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                                  int32_t max_context_len, float scale,
+                                  int32_t shared_prefix_tokens, int32_t partition_tokens,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                                  pa_dtype dtype, void* stream);
+
+/*
  * Attention of several query tokens per sequence over the paged cache, causal
  * within the chunk: the query tokens of sequence s are q rows q_start[s] ..
  * q_start[s+1]-1 and are the LAST Tq = q_start[s+1] - q_start[s] tokens of its

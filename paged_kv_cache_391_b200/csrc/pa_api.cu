@@ -215,10 +215,12 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
                     int32_t group_size, int32_t head_dim, int32_t block_size,
                     int64_t num_blocks, int32_t max_context_len, float scale,
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
-                    int32_t* dev_error, pa_dtype dtype, void* stream, bool persistent = false) {
+                    int32_t* dev_error, pa_dtype dtype, void* stream, bool persistent = false,
+                    int32_t shared_tokens = 0) {
   if (num_seqs < 0 || num_q_heads < 1 || group_size < 1 || num_blocks < 1 ||
       max_context_len < 0 || partition_tokens < 0 || !valid_dtype(dtype) || !isfinite(scale) ||
-      num_q_tokens < 0 || max_query_len < 0)
+      num_q_tokens < 0 || max_query_len < 0 || shared_tokens < 0 ||
+      shared_tokens > max_context_len)
     return PA_ERR_INVALID_ARG;
   if (block_size != PA_BLOCK_SIZE || (head_dim != 64 && head_dim != 128) || group_size > 16 ||
       num_q_heads % group_size != 0 || partition_tokens % PA_BLOCK_SIZE != 0)
@@ -293,6 +295,7 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   a.plan = nullptr;
   a.chunk_items = nullptr;
   a.chunk_plan = nullptr;
+  a.first_part = 0;
   if (persistent) {
     char* tail = static_cast<char*>(workspace) + need;
     a.items = reinterpret_cast<uint32_t*>(tail);
@@ -321,6 +324,22 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
     cudaError_t e = pa::launch_prefill_tc(a, tm_q, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = pa::launch_reduce(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : cuda_fail(e);
+  }
+  // A prefix shared by every sequence: its whole partitions (at least two,
+  // and not the last one) as one tcgen05 contraction over all sequences'
+  // queries, the rest by the decode kernel, the reduce over both.
+  if (!q_start && shared_tokens > 0 && parts > 2) {
+    const int64_t pp = shared_tokens / a.part_tokens;
+    a.first_part = (int32_t)(pp < parts - 1 ? pp : parts - 1);
+    if (a.first_part >= 2 && pa::prefill_tc_shared_supported(a)) {
+      CUtensorMap tm_q;
+      st = encode_query_map(&tm_q, q, num_q_tokens, num_q_heads, head_dim, group_size, dtype);
+      if (st != PA_OK) return st;
+      cudaError_t e = pa::launch_prefill_tc_shared(a, tm_q, static_cast<cudaStream_t>(stream));
+      if (e == cudaSuccess) e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
+      return e == cudaSuccess ? PA_OK : cuda_fail(e);
+    }
+    a.first_part = 0;
   }
   cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e);
@@ -355,6 +374,21 @@ pa_status pa_decode_persistent(void* out, const void* q, const void* k_cache,
                    block_table_stride, context_lens, num_seqs, num_q_heads, group_size, head_dim,
                    block_size, num_blocks, max_context_len, scale, partition_tokens, workspace,
                    workspace_bytes, dev_error, dtype, stream, true);
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  int32_t block_table_stride, const int32_t* context_lens,
+                                  int32_t num_seqs, int32_t num_q_heads, int32_t group_size,
+                                  int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                                  int32_t max_context_len, float scale,
+                                  int32_t shared_prefix_tokens, int32_t partition_tokens,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                                  pa_dtype dtype, void* stream) {
+  return attention(out, q, nullptr, num_seqs, 1, k_cache, v_cache, block_tables,
+                   block_table_stride, context_lens, num_seqs, num_q_heads, group_size, head_dim,
+                   block_size, num_blocks, max_context_len, scale, partition_tokens, workspace,
+                   workspace_bytes, dev_error, dtype, stream, false, shared_prefix_tokens);
 }
 
 pa_status pa_prefill_chunk(void* out, const void* q, const int32_t* q_start,

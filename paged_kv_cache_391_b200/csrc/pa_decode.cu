@@ -491,7 +491,8 @@ __global__ void __launch_bounds__(kThreads)
                             const int32_t* __restrict__ block_tables, int bt_stride,
                             const int32_t* __restrict__ context_lens, int num_q_heads, int group,
                             int64_t num_blocks, int max_context_len, float scale_log2,
-                            int part_blocks, int max_parts, int32_t* __restrict__ dev_error) {
+                            int part_blocks, int max_parts, int32_t* __restrict__ dev_error,
+                            int first_part) {
   using SM = DecodeSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -501,12 +502,31 @@ __global__ void __launch_bounds__(kThreads)
                       q,            q_start,   num_q_tokens, max_query_len, block_tables,
                       bt_stride,    context_lens, num_q_heads, group,       num_blocks,
                       max_context_len, scale_log2, part_blocks, max_parts,  dev_error};
-  const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x;
+  // first_part > 0 (decode only): the partitions below it, the shared
+  // prefix's, were computed by another kernel.
+  const int part = kMulti ? (int)(blockIdx.x % (unsigned)max_parts) : (int)blockIdx.x + first_part;
   const int qtile = kMulti ? (int)(blockIdx.x / (unsigned)max_parts) : 0;
   // Launched as a programmatic dependent: the CTA is resident when the
   // previous kernel ends, and waits for it before any read (empty
   // partitions then exit before setting up barriers).
   griddep_wait();
+  if (!kMulti && first_part > 0 && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32 &&
+      dev_error) {
+    // The prefix partitions assumed every sequence's table to start with
+    // sequence 0's first first_part * part_blocks entries and its context to
+    // cover them: a sequence for which that is false is counted (once; its
+    // output is then not its attention).
+    const int s = blockIdx.z, lane = threadIdx.x;
+    const int pre = first_part * part_blocks;
+    bool bad = false;
+    if (lane == 0) {
+      const int L = context_lens[s];
+      bad = L < pre * 16 || L > max_context_len;
+    }
+    const int32_t* row = block_tables + (size_t)s * bt_stride;
+    for (int i = lane; i < pre && s > 0; i += 32) bad |= row[i] != block_tables[i];
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicAdd(dev_error, 1);
+  }
   uint32_t ring = 0;
   (void)attend_item<T, D, kTwoRows, kMulti>(A, smem, bars, part, blockIdx.y, blockIdx.z, qtile,
                                             true, ring);
@@ -905,12 +925,15 @@ static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
   auto kern = decode_partition_kernel<T, D, kTwoRows, kMulti>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((int64_t)a.max_parts * a.max_qtiles), a.num_kv_heads, a.num_seqs);
+  // first_part (decode only) > 0: partitions from first_part on
+  const int64_t parts = (int64_t)a.max_parts - (kMulti ? 0 : a.first_part);
+  dim3 grid((unsigned)(parts * a.max_qtiles), a.num_kv_heads, a.num_seqs);
   e = launch_pdl(kern, grid, dim3(kThreads), SM::kAlloc, stream, a.tm_k, a.tm_v,
                  static_cast<T*>(a.out), a.part_o, a.part_lse, static_cast<const T*>(a.q),
                  a.q_start, a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride,
                  a.context_lens, a.num_q_heads, a.group, a.num_blocks, a.max_context_len,
-                 a.scale_log2, a.part_blocks, a.max_parts, a.dev_error);
+                 a.scale_log2, a.part_blocks, a.max_parts, a.dev_error,
+                 kMulti ? 0 : a.first_part);
   if (e != cudaSuccess) return e;
   return launch_reduce_typed<T, D>(a, stream);
 }

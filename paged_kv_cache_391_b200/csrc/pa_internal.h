@@ -44,6 +44,10 @@ struct DecodeLaunch {
   // {sequence, pair * max_parts + partition}, then [0] = items listed
   uint2* chunk_items;
   int32_t* chunk_plan;
+  // Decode with a shared prefix (pa_decode_shared_prefix): partitions below
+  // first_part are computed by the tcgen05 kernel over all sequences at once;
+  // the decode kernel starts at first_part. 0 otherwise.
+  int32_t first_part;
 };
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
@@ -67,6 +71,15 @@ bool prefill_tc_eligible(int32_t head_dim, int32_t group, int32_t max_query_len,
 int64_t prefill_tc_max_items(int32_t num_seqs, int32_t max_query_len, int32_t group,
                              int64_t parts);
 cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q, cudaStream_t stream);
+
+// The shared prefix's partitions [0, a.first_part) of every sequence on the
+// tcgen05 chunk kernel: the sequences' query tokens (one each, rows of q) as
+// the query tokens of one sequence whose context is the first
+// a.first_part * a.part_tokens keys of sequence 0's table, without a causal
+// mask, each partition's result written as the decode's fp32 partials.
+cudaError_t launch_prefill_tc_shared(const DecodeLaunch& a, const CUtensorMap& tm_q,
+                                     cudaStream_t stream);
+bool prefill_tc_shared_supported(const DecodeLaunch& a);
 
 // Records a CUDA error for pa_last_cuda_error() and returns PA_ERR_CUDA.
 pa_status record_cuda_error(cudaError_t e);

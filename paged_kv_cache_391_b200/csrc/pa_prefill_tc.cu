@@ -120,6 +120,7 @@ struct ChunkItem {
   int seq, kvh, part, qtile;  // qtile: the pair's first tile
   int L, q0, Tq, t0, n_parts, key_begin, key_end, n_steps;
   bool skip;                  // no rows or no keys of this item exist
+  bool causal;                // query token t sees keys up to L - Tq + t (else all L)
   int err_count;              // argument errors this item counts (its first item only)
 };
 
@@ -127,7 +128,8 @@ __device__ __forceinline__ ChunkItem chunk_item(int seq, int kvh, int part, int 
                                                 const int32_t* __restrict__ q_start,
                                                 int num_q_tokens, int max_query_len,
                                                 const int32_t* __restrict__ context_lens,
-                                                int group, int max_context_len, int part_blocks) {
+                                                int group, int max_context_len, int part_blocks,
+                                                int shared_L) {
   ChunkItem it;
   it.seq = seq;
   it.kvh = kvh;
@@ -135,6 +137,26 @@ __device__ __forceinline__ ChunkItem chunk_item(int seq, int kvh, int part, int 
   it.qtile = qtile;
   it.err_count = 0;
   it.skip = false;
+  it.causal = shared_L < 0;
+  if (shared_L >= 0) {
+    // A shared prefix: every row of q (one query token per sequence) sees
+    // all shared_L keys of sequence 0's table (checked by the host and the
+    // decode kernel), no mask.
+    const int tok_per_tile = kRows / group;
+    it.seq = 0;
+    it.L = shared_L;
+    it.q0 = 0;
+    it.Tq = num_q_tokens;
+    it.t0 = qtile * tok_per_tile;
+    const int nblk = (shared_L + 15) / 16;
+    it.n_parts = nblk > 0 ? (nblk + part_blocks - 1) / part_blocks : 1;
+    it.key_begin = part * part_blocks * 16;
+    it.key_end = min((part + 1) * part_blocks * 16, shared_L);
+    it.skip = it.t0 >= it.Tq || part >= it.n_parts;
+    it.n_steps = !it.skip && it.key_end > it.key_begin
+                     ? (it.key_end - it.key_begin + kKeys - 1) / kKeys : 0;
+    return it;
+  }
   const bool counts = part == 0 && kvh == 0 && qtile == 0;
   int L = context_lens[seq];
   if (L < 0 || L > max_context_len) {
@@ -194,7 +216,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                       int64_t num_blocks, int max_context_len, float scale_log2,
                       int part_blocks, int max_parts, int32_t* __restrict__ dev_error,
                       const uint2* __restrict__ items, int32_t* __restrict__ plan,
-                      int num_kv_heads) {
+                      int num_kv_heads, int shared_L) {
   using E = Elem<T>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
@@ -238,7 +260,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       qtile = (int)(pi.y / (unsigned)max_parts) * kTiles;
     }
     return chunk_item(seq, kvh, part, qtile, q_start, num_q_tokens, max_query_len,
-                      context_lens, group, max_context_len, part_blocks);
+                      context_lens, group, max_context_len, part_blocks, shared_L);
   };
   const bool persistent = plan != nullptr;
   if (persistent) {
@@ -539,13 +561,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const int tt0 = it.t0 + tile * tok_per_tile;       // first query token of the tile
       const int t = tt0 + r / group;                     // query token in the chunk
       const bool row_ok = t < Tq;
-      // the row's output: out row, and the partition (-1: one partition, direct)
+      // the row's output: out row, and the partition (-1: one partition,
+      // direct; a shared prefix's partitions are always partials)
       const size_t orow = (size_t)(it.q0 + t) * num_q_heads + it.kvh * group + r % group;
-      const int opart = it.n_parts == 1 ? -1 : it.part;
-      const int lim = L - Tq + (row_ok ? t : 0);         // last key this row may see
+      const int opart = it.n_parts == 1 && it.causal ? -1 : it.part;
+      // last key this row may see
+      const int lim = it.causal ? L - Tq + (row_ok ? t : 0) : L - 1;
       float m = -INFINITY, l = 0.f;                      // reference maximum (log2 units)
       // keys every row of the tile may see: up to the first row's causal limit
-      const int key_all = min(key_end, L - Tq + tt0 + 1);
+      const int key_all = it.causal ? min(key_end, L - Tq + tt0 + 1) : key_end;
       // Validity of the table entries of the step at key kb0 (a bit per cache
       // block), loaded one step ahead so the table reads never wait in the loop.
       auto bad_blocks = [&](int kb0) {
@@ -863,7 +887,7 @@ cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q,
           tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, a.q_start,
           a.num_q_tokens, a.max_query_len, a.block_tables, a.bt_stride, a.context_lens,
           a.num_q_heads, a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
-          a.max_parts, a.dev_error, nullptr, nullptr, a.num_kv_heads);
+          a.max_parts, a.dev_error, nullptr, nullptr, a.num_kv_heads, -1);
       return cudaGetLastError();
     }
     // Longest first: the plan kernel lists the items and zeroes the work
@@ -899,7 +923,38 @@ cudaError_t launch_prefill_tc(const DecodeLaunch& a, const CUtensorMap& tm_q,
                               a.group, a.num_blocks, a.max_context_len, a.scale_log2,
                               a.part_blocks, a.max_parts, a.dev_error,
                               static_cast<const uint2*>(a.chunk_items),
-                              a.chunk_plan, a.num_kv_heads);
+                              a.chunk_plan, a.num_kv_heads, -1);
+  };
+  return a.bf16 ? run((__nv_bfloat16*)nullptr) : run((__half*)nullptr);
+}
+
+bool prefill_tc_shared_supported(const DecodeLaunch& a) {
+  const int g = a.group;
+  return !a.q_start && a.head_dim == kD && (g == 1 || g == 2 || g == 4 || g == 8 || g == 16) &&
+         (int64_t)a.num_q_tokens * g >= 64 && a.part_tokens % kKeys == 0 && a.first_part >= 1 &&
+         a.first_part < a.max_parts && a.part_o && a.part_lse;
+}
+
+cudaError_t launch_prefill_tc_shared(const DecodeLaunch& a, const CUtensorMap& tm_q,
+                                     cudaStream_t stream) {
+  auto run = [&](auto* tag) -> cudaError_t {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    auto kern = prefill_tc_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    // one virtual sequence: all rows of q as its query tokens; its items are
+    // (tile pair, partition < first_part, KV head), grid order
+    const int64_t qtiles = ((int64_t)a.num_q_tokens * a.group + kRows - 1) / kRows;
+    const int64_t pairs = (qtiles + kTiles - 1) / kTiles;
+    const int shared_L = a.first_part * a.part_tokens;
+    dim3 grid((unsigned)((int64_t)a.max_parts * pairs), a.num_kv_heads, 1);
+    kern<<<grid, kThreadsTc, kSmemAlloc, stream>>>(
+        tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, nullptr,
+        a.num_q_tokens, a.num_q_tokens, a.block_tables, a.bt_stride, nullptr, a.num_q_heads,
+        a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks, a.max_parts,
+        a.dev_error, nullptr, nullptr, a.num_kv_heads, shared_L);
+    return cudaGetLastError();
   };
   return a.bf16 ? run((__nv_bfloat16*)nullptr) : run((__half*)nullptr);
 }

@@ -29,7 +29,7 @@ EXPORTS = ("pa_write_kv", "pa_decode_workspace_size", "pa_decode", "pa_copy_bloc
            "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_slots", "pa_bm_append_slots",
            "pa_bm_block_tables", "pa_bm_get_stats", "pa_bm_refcount", "pa_prefill_chunk",
            "pa_decode_persistent_workspace_size", "pa_decode_persistent", "pa_read_probe",
-           "pa_prefill_chunk_workspace_size")
+           "pa_prefill_chunk_workspace_size", "pa_decode_shared_prefix")
 PA_STATIC_WORKSPACE_BYTES = 32 << 20
 
 _lock = threading.Lock()
@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.pa_decode_persistent_workspace_size.restype = sz
             L.pa_decode_persistent.argtypes = L.pa_decode.argtypes
             L.pa_decode_persistent.restype = ctypes.c_int
+            L.pa_decode_shared_prefix.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32,
+                                                  i64, i32, ctypes.c_float, i32, i32, P, sz, P,
+                                                  ctypes.c_int, P]
+            L.pa_decode_shared_prefix.restype = ctypes.c_int
             L.pa_prefill_chunk.argtypes = [P, P, P, i32, i32, P, P, P, i32, P, i32, i32, i32,
                                            i32, i32, i64, i32, ctypes.c_float, i32, P, sz, P,
                                            ctypes.c_int, P]
@@ -200,11 +204,14 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
            block_tables: torch.Tensor, context_lens: torch.Tensor, *, scale: float,
            max_context_len: int, partition_tokens: int = 512,
            workspace: torch.Tensor | None = None, dev_error: torch.Tensor | None = None,
-           stream=None, persistent: bool = False) -> torch.Tensor:
+           stream=None, persistent: bool = False,
+           shared_prefix_tokens: int = 0) -> torch.Tensor:
     """Paged decode attention: ``out [S, H_q, D] = attention(q, paged K/V)``.
     ``persistent=True`` runs pa_decode_persistent (work-queue schedule, the
     same result bit for bit); its workspace comes from
-    ``alloc_workspace(..., persistent=True)``."""
+    ``alloc_workspace(..., persistent=True)``. ``shared_prefix_tokens > 0``
+    runs pa_decode_shared_prefix: every sequence starts with that many tokens
+    in sequence 0's blocks."""
     S, Hq, D = q.shape
     NB, Hkv = k_cache.shape[:2]
     assert out.shape == q.shape and out.dtype == q.dtype == k_cache.dtype == v_cache.dtype
@@ -217,6 +224,16 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
         workspace = alloc_workspace(S, Hq, D, max_context_len, partition_tokens, q.device,
                                     persistent)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if shared_prefix_tokens:
+        if persistent:
+            raise ValueError("shared_prefix_tokens and persistent do not combine")
+        st = lib().pa_decode_shared_prefix(
+            _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            block_tables.shape[1], _ptr(context_lens), S, Hq, Hq // Hkv, D, PA_BLOCK_SIZE, NB,
+            int(max_context_len), float(scale), int(shared_prefix_tokens), int(partition_tokens),
+            _ptr(workspace), ws_bytes, _ptr(dev_error), _dtype_code(q), _stream(stream, q.device))
+        _check(st, "pa_decode_shared_prefix")
+        return out
     fn = lib().pa_decode_persistent if persistent else lib().pa_decode
     st = fn(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
             block_tables.shape[1], _ptr(context_lens), S, Hq, Hq // Hkv, D, PA_BLOCK_SIZE, NB,

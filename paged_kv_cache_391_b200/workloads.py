@@ -349,7 +349,9 @@ def gqa(seed: int = 393, batch: int = 256, sigma: float = 1.0) -> DecodeWorkload
 
 
 def shared_prefix(seed: int = 394, num_seqs: int = 100, prefix: int = 5000,
-                  suffix_lo: int = 16, suffix_hi: int = 512) -> DecodeWorkload:
+                  suffix_lo: int = 16, suffix_hi: int = 512, num_q_heads: int = 32,
+                  num_kv_heads: int = 8, head_dim: int = 128,
+                  dtype: str = "bf16") -> DecodeWorkload:
     """100 sequences whose tables share one 5000-token prefix (313 blocks, the
     last one holding 8 tokens) plus unique suffixes uniform in [16, 512]
     tokens; H_q = 32, H_kv = 8, D = 128, bf16 ("KV Cache Sharing
@@ -363,7 +365,7 @@ def shared_prefix(seed: int = 394, num_seqs: int = 100, prefix: int = 5000,
     cached, the copy's free slots first. The step writes each sequence's
     newest token and decodes; the 312 full prefix blocks stay shared and
     unchanged. The fork itself happened before this step, so the step has no
-    copy pairs."""
+    copy pairs. (Other head counts, head sizes and dtypes for tests.)"""
     rng = np.random.default_rng(seed)
     suf = rng.integers(suffix_lo, suffix_hi, size=num_seqs, endpoint=True)
     n_prefix_blocks = blocks_needed(prefix)
@@ -389,8 +391,8 @@ def shared_prefix(seed: int = 394, num_seqs: int = 100, prefix: int = 5000,
     fills += [(int(p), BLOCK_SIZE) for p in shared[:full]]
     if tail:
         fills.append((int(shared[full]), tail))
-    w = _build("shared_prefix", "bf16", 32, 8, 128, 512, seed, rng, tables, fills, lens, nb,
-               writes, [],
+    w = _build("shared_prefix", dtype, num_q_heads, num_kv_heads, head_dim, 512, seed, rng,
+               tables, fills, lens, nb, writes, [],
                {"prefix": prefix, "shared_blocks": full,
                 "partial_prefix_block": int(shared[full]) if tail else -1,
                 "fork_pairs": forks})

@@ -168,6 +168,31 @@ def test_decode_persistent_rejects_on_the_host(L, kw, status):
     assert _decode_persistent(L, **kw) == status
 
 
+def _decode_shared(L, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, stride=4, cl=FAKE, S=2, Hq=8, g=4, D=128,
+             bs=16, NB=10, max_ctx=64, scale=0.1, shared=0, P=512, ws=None, ws_bytes=0, err=None,
+             dt=1)
+    a.update(kw)
+    return L.pa_decode_shared_prefix(a["out"], a["q"], a["k"], a["v"], a["bt"], a["stride"],
+                                     a["cl"], a["S"], a["Hq"], a["g"], a["D"], a["bs"], a["NB"],
+                                     a["max_ctx"], ctypes.c_float(a["scale"]), a["shared"],
+                                     a["P"], a["ws"], a["ws_bytes"], a["err"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(shared=-1), pa.PA_ERR_INVALID_ARG),
+    (dict(shared=65), pa.PA_ERR_INVALID_ARG),                 # longer than max_context_len
+    (dict(g=3), pa.PA_ERR_UNSUPPORTED),
+    (dict(out=None, shared=32), pa.PA_ERR_INVALID_ARG),
+    (dict(max_ctx=2048, stride=128, shared=1536), pa.PA_ERR_INVALID_ARG),  # needs a workspace
+    (dict(max_ctx=2048, stride=128, shared=1536, ws=FAKE, ws_bytes=100),
+     pa.PA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(S=0, shared=32), pa.PA_OK),                         # nothing to do
+])
+def test_decode_shared_prefix_rejects_on_the_host(L, kw, status):
+    assert _decode_shared(L, **kw) == status
+
+
 def _prefill(L, **kw):
     a = dict(out=FAKE, q=FAKE, qs=FAKE, nq=8, maxq=4, k=FAKE, v=FAKE, bt=FAKE, stride=4, cl=FAKE,
              S=2, Hq=8, g=4, D=128, bs=16, NB=10, max_ctx=64, scale=0.1, P=512, ws=None,

@@ -33,6 +33,18 @@ def _make(mode):
                              max_query_len=mq, max_context_len=w.max_context_len,
                              partition_tokens=d.P, workspace=ws, dev_error=d.err)
         return w, d, attend
+    if mode == "shared":
+        w = W.shared_prefix(num_seqs=24, prefix=2100, suffix_hi=300)
+        d = DeviceStep(w, 512)
+        ws = pa.alloc_workspace(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, 512,
+                                "cuda")
+        shared = int(w.notes["shared_blocks"]) * pa.PA_BLOCK_SIZE
+
+        def attend(out):
+            pa.decode(out, d.q, d.k_cache, d.v_cache, d.bt, d.cl, scale=w.scale,
+                      max_context_len=w.max_context_len, partition_tokens=512, workspace=ws,
+                      dev_error=d.err, shared_prefix_tokens=shared)
+        return w, d, attend
     w = W.tiny() if mode == "tiny" else W.gqa(batch=12)
     d = DeviceStep(w, partition_tokens=16 if mode == "tiny" else None)
     persistent = mode == "persistent"
@@ -46,7 +58,7 @@ def _make(mode):
     return w, d, attend
 
 
-@pytest.mark.parametrize("mode", ["tiny", "grid", "persistent", "chunk"])
+@pytest.mark.parametrize("mode", ["tiny", "grid", "persistent", "chunk", "shared"])
 def test_step_replays_as_a_cuda_graph(mode):
     w, d, attend = _make(mode)
 
