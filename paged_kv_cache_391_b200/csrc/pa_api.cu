@@ -296,6 +296,7 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
   a.chunk_items = nullptr;
   a.chunk_plan = nullptr;
   a.first_part = 0;
+  a.shared_tm_q = nullptr;
   if (persistent) {
     char* tail = static_cast<char*>(workspace) + need;
     a.items = reinterpret_cast<uint32_t*>(tail);
@@ -335,8 +336,8 @@ pa_status attention(void* out, const void* q, const int32_t* q_start, int32_t nu
       CUtensorMap tm_q;
       st = encode_query_map(&tm_q, q, num_q_tokens, num_q_heads, head_dim, group_size, dtype);
       if (st != PA_OK) return st;
-      cudaError_t e = pa::launch_prefill_tc_shared(a, tm_q, static_cast<cudaStream_t>(stream));
-      if (e == cudaSuccess) e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
+      a.shared_tm_q = &tm_q;  // the decode's launch runs the prefix kernel after its own
+      cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
       return e == cudaSuccess ? PA_OK : cuda_fail(e);
     }
     a.first_part = 0;

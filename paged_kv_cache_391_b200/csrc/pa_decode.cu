@@ -527,6 +527,9 @@ __global__ void __launch_bounds__(kThreads)
     for (int i = lane; i < pre && s > 0; i += 32) bad |= row[i] != block_tables[i];
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicAdd(dev_error, 1);
   }
+  // With a shared prefix the next kernel, the prefix's partitions, reads
+  // nothing this one writes: it may start on the SMs this grid leaves free.
+  if (!kMulti && first_part > 0) griddep_launch_dependents();
   uint32_t ring = 0;
   (void)attend_item<T, D, kTwoRows, kMulti>(A, smem, bars, part, blockIdx.y, blockIdx.z, qtile,
                                             true, ring);
@@ -935,6 +938,12 @@ static cudaError_t launch_typed(const DecodeLaunch& a, cudaStream_t stream) {
                  a.scale_log2, a.part_blocks, a.max_parts, a.dev_error,
                  kMulti ? 0 : a.first_part);
   if (e != cudaSuccess) return e;
+  if (!kMulti && a.first_part > 0 && a.shared_tm_q) {
+    // the shared prefix's partitions, overlapping this kernel's end; the
+    // reduce after them waits for both
+    e = launch_prefill_tc_shared(a, *a.shared_tm_q, stream);
+    if (e != cudaSuccess) return e;
+  }
   return launch_reduce_typed<T, D>(a, stream);
 }
 

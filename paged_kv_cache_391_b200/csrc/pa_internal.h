@@ -46,8 +46,11 @@ struct DecodeLaunch {
   int32_t* chunk_plan;
   // Decode with a shared prefix (pa_decode_shared_prefix): partitions below
   // first_part are computed by the tcgen05 kernel over all sequences at once;
-  // the decode kernel starts at first_part. 0 otherwise.
+  // the decode kernel starts at first_part. 0 otherwise. shared_tm_q (the
+  // query map of that kernel) set: the decode's launch makes it, between the
+  // decode kernel and the reduce.
   int32_t first_part;
+  const CUtensorMap* shared_tm_q;
 };
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);

@@ -268,7 +268,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   } else {
     const ChunkItem it = item_of(kGridItem);
     if (tid == 0 && it.err_count && dev_error) atomicAdd(dev_error, it.err_count);
-    if (it.skip) return;  // uniform over the CTA, before any barrier
+    if (it.skip) {  // uniform over the CTA, before any barrier
+      if (shared_L >= 0) griddep_wait();  // see the end of the kernel
+      return;
+    }
   }
 
   // ---- set-up: barriers (thread 0), TMEM (warp 0)
@@ -760,6 +763,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
+  // A shared prefix's partitions run as a programmatic dependent of the
+  // decode kernel that covers the other partitions, overlapping its end (the
+  // two write disjoint partials; the inputs were complete before that kernel
+  // started). This grid ends only after that one, so the reduce launched
+  // after this grid, which waits for it, sees both.
+  if (shared_L >= 0) griddep_wait();
 }
 
 // Longest-first order of the chunk kernel's work: the CTAs of a grid start in
@@ -948,13 +957,24 @@ cudaError_t launch_prefill_tc_shared(const DecodeLaunch& a, const CUtensorMap& t
     const int64_t qtiles = ((int64_t)a.num_q_tokens * a.group + kRows - 1) / kRows;
     const int64_t pairs = (qtiles + kTiles - 1) / kTiles;
     const int shared_L = a.first_part * a.part_tokens;
-    dim3 grid((unsigned)((int64_t)a.max_parts * pairs), a.num_kv_heads, 1);
-    kern<<<grid, kThreadsTc, kSmemAlloc, stream>>>(
-        tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out), a.part_o, a.part_lse, nullptr,
-        a.num_q_tokens, a.num_q_tokens, a.block_tables, a.bt_stride, nullptr, a.num_q_heads,
-        a.group, a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks, a.max_parts,
-        a.dev_error, nullptr, nullptr, a.num_kv_heads, shared_L);
-    return cudaGetLastError();
+    // a programmatic dependent of the decode kernel launched before it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)a.max_parts * pairs), a.num_kv_heads, 1);
+    cfg.blockDim = dim3(kThreadsTc);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tm_q, a.tm_k, a.tm_v, static_cast<T*>(a.out),
+                              a.part_o, a.part_lse, static_cast<const int32_t*>(nullptr),
+                              a.num_q_tokens, a.num_q_tokens, a.block_tables, a.bt_stride,
+                              static_cast<const int32_t*>(nullptr), a.num_q_heads, a.group,
+                              a.num_blocks, a.max_context_len, a.scale_log2, a.part_blocks,
+                              a.max_parts, a.dev_error, static_cast<const uint2*>(nullptr),
+                              static_cast<int32_t*>(nullptr), a.num_kv_heads, shared_L);
   };
   return a.bf16 ? run((__nv_bfloat16*)nullptr) : run((__half*)nullptr);
 }
