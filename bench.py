@@ -64,9 +64,10 @@ def parse():
     ap.add_argument("--workload", default="long", choices=list(WORKLOAD_TEXT),
                     help="the headline workload (default: the long-context config, the "
                          "largest that fits one GPU)")
-    ap.add_argument("--also", default="gqa",
+    ap.add_argument("--also", default="gqa,chunked_prefill,shared_prefix:shared",
                     help="comma-separated workloads measured in the same run and reported "
-                         "under 'also' (empty: none)")
+                         "under 'also' (empty: none); workload:scheduler picks that "
+                         "workload's scheduler")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling only)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--op", default="step", choices=["step", "swap", "blockmgr"],
@@ -913,9 +914,17 @@ def main():
                                 device_id=device)
 
     names = [args.workload] + [n for n in args.also.split(",") if n and n != args.workload]
+    entry_args = {}
     for n in names:
-        if n not in WORKLOAD_TEXT:
+        wl, _, sched = n.partition(":")
+        if wl not in WORKLOAD_TEXT or (sched and sched not in ("grid", "persistent", "shared")):
             raise SystemExit(f"unknown workload {n}")
+        a = args
+        if sched:
+            import copy
+            a = copy.copy(args)
+            a.scheduler = sched
+        entry_args[n] = (wl, a)
     records = {}
     ceiling = None
     with ClockSampler(device.index if device.index is not None else 0) as clocks:
@@ -925,7 +934,8 @@ def main():
         if not args.no_read_probe:
             ceiling = read_ceiling(device)
         for i, name in enumerate(names):
-            res = run_gpu(args, name, rank, world, device, probe_buf=probe_buf)
+            wl, a = entry_args[name]
+            res = run_gpu(a, wl, rank, world, device, probe_buf=probe_buf)
             agg = reduce_over_ranks(res, world, device)
             records[name] = (res, agg)
             if i > 0:                  # keep only the headline's pools (the CPU leg reads them)
@@ -933,7 +943,8 @@ def main():
             torch.cuda.empty_cache()
         del probe_buf
     head_res, head_agg = records[args.workload]
-    rec = workload_record(args.workload, head_res, head_agg, args, world, ceiling)
+    rec = workload_record(args.workload, head_res, head_agg, entry_args[args.workload][1], world,
+                          ceiling)
     line = {
         "metric": METRIC,
         "value": rec["value"],
@@ -954,7 +965,8 @@ def main():
         line["read_ceiling"] = ceiling
     also = {}
     for name in names[1:]:
-        r = workload_record(name, *records[name], args, world, ceiling)
+        wl, a = entry_args[name]
+        r = workload_record(wl, *records[name], a, world, ceiling)
         also[name] = r
     if also:
         line["also"] = also
