@@ -838,6 +838,28 @@ def workload_record(name, res, agg, args, world, ceiling) -> dict:
                                     f"kernel's CTA shape")
     if traffic and not tensor_bound:
         roof["dram_gbs"] = round(traffic / (att_ms / 1e3) / 1e9, 1)
+    shared = res.get("shared_tokens", 0)
+    if shared and not tensor_bound:
+        # pa_decode_shared_prefix reads the shared partitions' K/V once for all
+        # sequences: its roofline figure counts those bytes once (the logical
+        # figure, each sequence's whole context, stays in kv_gbs and value)
+        P = w.partition_tokens
+        parts = -(-w.max_context_len // P) if P else 1
+        first = min(shared // P, parts - 1) if P else 0
+        if first >= 2:
+            per_seq = first * P * w.num_kv_heads * w.head_dim * 2 * w.elem_bytes()
+            distinct = sb["decode"] - (w.num_seqs - 1) * per_seq
+            d_ach = distinct / (att_ms / 1e3) / 1e9
+            roof["achieved"] = round(d_ach, 1)
+            roof["frac"] = round(d_ach / peak, 4)
+            roof["algorithmic_bytes_per_launch"] = int(distinct)
+            roof["bytes_note"] = ("distinct K/V bytes: the shared partitions counted once "
+                                  f"({first} x {P} tokens), the rest per sequence; "
+                                  "kv_gbs counts every sequence's whole context")
+            roof["traffic"] = roof["traffic_ratio"] = None
+            if ceiling:
+                roof["frac_read"] = round(d_ach / ceiling["gbs"], 4)
+                roof["frac_read_paged"] = round(d_ach / ceiling["scattered_tiles_gbs"], 4)
     rec = {
         "value": round(value, 2), "unit": "GB/s", "ms_per_step": round(elapsed_ms / K, 5),
         "seq_steps_per_s": round(agg["seqs"] * K / (elapsed_ms / 1e3), 1),
