@@ -847,7 +847,7 @@ def workload_record(name, res, agg, args, world, ceiling) -> dict:
         parts = -(-w.max_context_len // P) if P else 1
         first = min(shared // P, parts - 1) if P else 0
         if first >= 2:
-            per_seq = first * P * w.num_kv_heads * w.head_dim * 2 * w.elem_bytes()
+            per_seq = first * P * w.num_kv_heads * w.head_dim * 2 * w.elem_bytes
             distinct = sb["decode"] - (w.num_seqs - 1) * per_seq
             d_ach = distinct / (att_ms / 1e3) / 1e9
             roof["achieved"] = round(d_ach, 1)

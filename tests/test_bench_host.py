@@ -108,3 +108,32 @@ def test_last_block_waste():
     r = bench.waste_stats(w)
     assert r["mean_slots_per_seq"] == 7.75
     assert r["pct_of_allocated_slots"] == round(100 * 31 / 96, 4)
+
+
+def test_shared_prefix_record_counts_the_shared_partitions_once():
+    """The bench record of the shared-prefix path (synthetic timings, no GPU):
+    the roofline's bytes are the distinct K/V bytes (9 shared partitions of
+    512 tokens once, the rest per sequence); the logical rate stays in
+    kv_gbs; the record is plain JSON."""
+    import argparse
+    import json
+    w = bench.make_workload("shared_prefix", None)
+    res = {"w": w, "sus_reps": 10, "persistent": False, "shared_tokens": 4992, "tc_path": False,
+           "copy_pairs": 0, "copy_what": "", "short_reps": 200, "rounds": 1, "launches": 4,
+           "e2e": None, "att_reps": 20}
+    agg = {"ms": 1.3, "att_ms": 0.06, "kv": w.kv_bytes(), "sus_ms": 0.07, "seqs": w.num_seqs,
+           "write_ms": 0.004, "copy_ms": 0.004, "errors": 0, "e2e_ms": 1.4}
+    args = argparse.Namespace(steps=20, batch=None, workload="long", sustain_seconds=3.0,
+                              scheduler="shared")
+    ceiling = {"gbs": 7100.0, "scattered_tiles_gbs": 6800.0, "bytes": 2 << 30,
+               "vector_loads_gbs": 7000.0, "bulk_copies_gbs": 7100.0}
+    rec = bench.workload_record("shared_prefix", res, agg, args, 1, ceiling)
+    roof = rec["roofline"]
+    per_seq = 9 * 512 * w.num_kv_heads * w.head_dim * 2 * 2
+    distinct = w.step_bytes()["decode"] - (w.num_seqs - 1) * per_seq
+    assert roof["algorithmic_bytes_per_launch"] == distinct
+    assert abs(roof["achieved"] - distinct / 0.06e-3 / 1e9) < 0.1
+    assert roof["kv_gbs"] > 5 * roof["achieved"]          # logical: every whole context
+    assert roof["bound"] == "hbm" and roof["traffic"] is None
+    assert "pa_decode_shared_prefix" in roof["kernel"]
+    json.dumps(rec)
