@@ -122,3 +122,24 @@ def test_full_size_shared_prefix_sampled():
     ref = oracle.decode(w.q[seqs], kc, vc, w.block_tables[seqs], w.context_lens[seqs], w.scale,
                         w.dtype)
     assert_decode_close(to_f64(out)[seqs], ref, "full-size shared prefix")
+
+
+def test_a_prefix_that_is_the_whole_context():
+    """Every context is exactly the 2,048 shared tokens: of its four 512-token
+    partitions the first three are shared and the last is left to the decode
+    kernel (it always keeps the longest context's last partition)."""
+    w = W.shared_prefix(num_seqs=24, prefix=2100, suffix_hi=300, seed=71)
+    d = DeviceStep(w, 512)
+    d.cache_ops()
+    L = 2048
+    cl = torch.full_like(d.cl, L)
+    out = torch.full_like(d.out, float("nan"))
+    d.err.zero_()
+    pa.decode(out, d.q, d.k_cache, d.v_cache, d.bt, cl, scale=w.scale, max_context_len=L,
+              partition_tokens=512, dev_error=d.err, shared_prefix_tokens=L)
+    torch.cuda.synchronize()
+    assert int(d.err.item()) == 0
+    kc, vc = oracle_caches_after_step(w)
+    ref = oracle.decode(w.q, kc, vc, w.block_tables, np.full(w.num_seqs, L, np.int32), w.scale,
+                        w.dtype)
+    assert_decode_close(to_f64(out), ref, "prefix = whole context")
