@@ -58,6 +58,22 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 
 
+def test_reference_arm_runs_on_rank_0_only():
+    """Launched by torchrun with N > 1, the reference arm's other ranks exit 0
+    at once and print nothing (rank 0 alone times the oracle)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "2", "--warmup", "1",
+                        "--cpu-seconds", "0.2"], capture_output=True, text=True, timeout=300,
+                       cwd=root, env=env)
+    assert r.returncode == 0, r.stderr
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
 def test_recorded_traffic_follows_the_kernel_sources():
     """A traffic figure is reported for a full-size workload only while the
     hash of its kernel family's sources matches the recorded one."""
